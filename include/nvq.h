@@ -1,0 +1,177 @@
+/*
+ * nvq.h -- C ABI of the phase-specialised quantized linear layers for B200 (sm_100a).
+ *
+ * Prefill: NVFP4 W4A4.  Activations and weights are quantized to NVFP4 by
+ * round-to-nearest: E2M1 4-bit codes in 16-element blocks along K, one E4M3
+ * scale per block and one FP32 scale per tensor (Mix-Quant page, gist.science,
+ * section 2 "hybrid precision strategy"; section 2.3: the prefill worker runs
+ * the NVFP4 W4A4 path).  The quantized operands feed a block-scaled GEMM on the
+ * tcgen05 tensor cores.
+ *
+ * Decode: W4A16.  BF16 activations at small batch multiply INT4 weights that
+ * carry one BF16 scale per group of 128 weights; the weights are reordered
+ * offline into the kernel's fragment order (MARLIN page, abeam.tech, sections
+ * "weight layout" and "overlapping memory and compute").
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no device memory and frees nothing.  Outputs are written in place.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on that stream; no call synchronises the host
+ *     except nvq_check_device_error().
+ *   - Matrices are row-major.  BF16 is IEEE bfloat16 stored as 16-bit words.
+ *   - Packed 4-bit codes: two per byte, the even-k element in the low nibble.
+ *   - The return value reports host-side validation and launch errors
+ *     (cudaGetLastError after launch).  Errors found on the device (a bounded
+ *     wait that ran out) set a library-wide device error word that
+ *     nvq_check_device_error() reads and clears.  No kernel traps.
+ *   - Pointers must be 16-byte aligned (NVQ_ERR_MISALIGNED otherwise).
+ */
+#ifndef NVQ_H_
+#define NVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVQ_OK = 0,
+  NVQ_ERR_INVALID_ARG = 1,        /* null pointer, negative size */
+  NVQ_ERR_UNSUPPORTED_SHAPE = 2,  /* shape outside the documented rules */
+  NVQ_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned */
+  NVQ_ERR_WORKSPACE = 4,          /* workspace missing or too small */
+  NVQ_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+  NVQ_ERR_DEVICE_TIMEOUT = 6      /* a kernel's bounded wait ran out */
+} nvq_status;
+
+/* Version of this ABI; bumped on any incompatible change. */
+int nvq_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* nvq_status_string(nvq_status s);
+
+/* Text describing the last failed call on this host thread (argument or CUDA
+ * error), or "" if none; owned by the library, valid until the next call. */
+const char* nvq_last_error_detail(void);
+
+/* Synchronises `stream`, then reads and clears the device error word.
+ * Returns NVQ_ERR_DEVICE_TIMEOUT if any kernel since the last check gave up on
+ * a bounded wait, NVQ_ERR_CUDA if the synchronisation failed, else NVQ_OK. */
+nvq_status nvq_check_device_error(void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * NVFP4 round-to-nearest quantization (Mix-Quant page, section 2: 16-element
+ * groups with a local scale plus a tensor-level scale, plain RTN).
+ *
+ *   t   = *tensor_scale_in if tensor_scale_in != NULL, else
+ *         1.0f if max|x| == 0, else fp32_RNE(max|x| / 2688)   (2688 = 6 * 448)
+ *   s_b = E4M3_RNE_satfinite(amax_b / (6 t))   for each 16-element block b
+ *   c   = sign(x) | E2M1_RNE_satfinite(|x| / (e4m3(s_b) t)), ties to the even
+ *         code; a block with s_b == 0 stores magnitude 0 (sign kept)
+ * Every rounding is decided on the exact real quotient (the same result as
+ * infinitely precise division followed by one rounding).
+ *
+ * x_bf16            [rows, K] BF16, row stride K elements.  Inputs are finite;
+ *                   non-finite values are outside the contract.
+ * rows              >= 0 (0 is a no-op that still writes tensor_scale_out = 1
+ *                   when tensor_scale_in == NULL).
+ * K                 > 0, K % 64 == 0.
+ * tensor_scale_in   NULL, or a device pointer to a caller-fixed positive finite
+ *                   FP32 t (a static activation scale).
+ * codes             [rows, K/2] bytes, written.
+ * scales            nvfp4_scales_bytes(rows, K) bytes, written in the tiled
+ *                   layout that the block-scaled MMA reads: 512-byte atoms of
+ *                   128 rows x 4 blocks, row r / block c of an atom at byte
+ *                   16*(r%32) + 4*((r%128)/32) + c, atoms K-fastest
+ *                   (atom index = (r/128)*(K/64) + kb/4).  Padding rows (rows
+ *                   up to the next multiple of 128) get zero scales.
+ * tensor_scale_out  device pointer, receives t (may alias tensor_scale_in).
+ * workspace         device scratch of nvfp4_quantize_workspace_bytes(rows, K)
+ *                   bytes (may be NULL when that is 0).
+ * ------------------------------------------------------------------------ */
+size_t nvfp4_scales_bytes(int64_t rows, int64_t K);
+size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K);
+nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K,
+                          const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,
+                          float* tensor_scale_out, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * NVFP4 W4A4 GEMM (Mix-Quant page, section 2.3: the prefill worker's W4A4 path).
+ *
+ *   Y[m, n] = bf16_RNE( t_x * t_w * sum_k (e4m3(sx[m, k/16]) e2m1(cx[m, k]))
+ *                                        * (e4m3(sw[n, k/16]) e2m1(cw[n, k])) )
+ * accumulated in FP32 on the tensor cores (tcgen05 block-scaled MMA, TMEM
+ * accumulators).  Operands are the outputs of nvfp4_quantize: X [M, K] and
+ * W [N, K] (nn.Linear layout), so Y = X W^T.
+ *
+ * x_codes [M, K/2], x_scales (tiled, nvfp4_scales_bytes(M, K)), t_x (device FP32)
+ * w_codes [N, K/2], w_scales (tiled, nvfp4_scales_bytes(N, K)), t_w (device FP32)
+ * y_bf16  [M, N] BF16, row stride N, written.
+ * Shape rules: M >= 0, N >= 8, N % 8 == 0, K >= 64, K % 64 == 0.
+ * ------------------------------------------------------------------------ */
+nvq_status nvfp4_gemm_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const float* t_x,
+                           const uint8_t* w_codes, const uint8_t* w_scales, const float* t_w,
+                           void* y_bf16, int64_t M, int64_t N, int64_t K, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * INT4 group-128 round-to-nearest weight quantization (MARLIN page: 4-bit
+ * weights with one scale per 128-weight group).
+ *
+ *   s[n, g] = bf16_RNE(amax(w[n, 128g : 128g+128]) / 7)
+ *   q       = clamp(RNE_half_even(w / s), -8, 7)   (0 when s == 0)
+ *   u       = q + 8, stored as nibbles, even k in the low nibble
+ * w_bf16 [N, K]; codes [N, K/2] bytes; scales_bf16 [N, K/128] BF16.
+ * Shape rules: N >= 0, K > 0, K % 128 == 0.
+ * ------------------------------------------------------------------------ */
+nvq_status int4_quantize(const void* w_bf16, int64_t N, int64_t K, uint8_t* codes,
+                         void* scales_bf16, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * Offline reorder of INT4 codes and group scales into the decode kernel's
+ * fragment order (MARLIN page, "weight layout": codes and scales are permuted
+ * ahead of time so each thread's loads are regular and dequantize straight
+ * into tensor-core fragment order).  A bijection: no byte is added or lost.
+ *
+ * Unit = 16 weight rows x one 128-wide group: 1024 code bytes at unit index
+ * (n/16)*(K/128) + k/128.  Inside a unit, 32-bit word 128h + 4lane + jj (h in
+ * {0,1}, lane = 4g + c in [0,32), jj in [0,4)) holds k16-step j = 4h + jj with
+ * nibble p (bits 4p..4p+3) at (row, k-in-group):
+ *   p=0 (g, 16j+2c)   p=4 (g, 16j+2c+1)   p=1 (g+8, 16j+2c)   p=5 (g+8, 16j+2c+1)
+ *   p=2 (g, 16j+2c+8) p=6 (g, 16j+2c+9)   p=3 (g+8, 16j+2c+8) p=7 (g+8, 16j+2c+9)
+ * Scales: 32 bytes per unit; 32-bit word g holds rows g (low) and g+8 (high).
+ *
+ * codes [N, K/2] (as written by int4_quantize), scales_bf16 [N, K/128]
+ * packed_codes N*K/2 bytes, packed_scales N*(K/128)*2 bytes, written.
+ * Shape rules: N % 16 == 0, K % 128 == 0.
+ * ------------------------------------------------------------------------ */
+nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int64_t N, int64_t K,
+                             uint8_t* packed_codes, void* packed_scales, void* stream);
+
+/* ------------------------------------------------------------------------ *
+ * W4A16 decode GEMM (MARLIN page: FP16/BF16 activations x INT4 weights with
+ * group-128 scales, streaming the weights asynchronously with an L2-sparing
+ * cache policy, dequantizing in registers next to the tensor-core MMAs).
+ *
+ *   Y[m, n] = bf16_RNE( sum_g s[n, g] * sum_{k in g} x[m, k] * (u[n, k] - 8) )
+ * with the inner sums accumulated in FP32 (the products x * (u - 8) are exact)
+ * and the group scale applied in FP32.
+ *
+ * x_bf16 [M, K] BF16; packed_codes / packed_scales from int4_pack_weights;
+ * y_bf16 [M, N] BF16, row stride N, written.
+ * workspace: w4a16_workspace_bytes(M, N, K) bytes of device scratch (split-K
+ * partial sums); may be NULL when that is 0.
+ * Shape rules: M >= 0, N % 16 == 0, K % 128 == 0.
+ * ------------------------------------------------------------------------ */
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
+nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const void* packed_scales,
+                      void* y_bf16, int64_t M, int64_t N, int64_t K,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVQ_H_ */

@@ -1,0 +1,185 @@
+"""Phase-specialised quantized linear layers for B200 (sm_100a).
+
+Thin Python binding of the C-ABI library ``libnvq.so`` (declared in
+``include/nvq.h``).  Every function here only marshals arguments: it allocates
+outputs with torch when the caller does not pass them, takes device pointers,
+and calls the library entry point of the same name on the current CUDA stream.
+All arithmetic runs in the library's CUDA kernels.  There is no CPU fallback:
+if the library or a GPU is missing, the calls raise.
+
+Prefill (Mix-Quant page, gist.science, section 2): ``nvfp4_quantize`` then
+``nvfp4_gemm_w4a4``.  Decode (MARLIN page, abeam.tech): ``int4_quantize`` and
+``int4_pack_weights`` offline, then ``w4a16_gemm``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnvq.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "nvq.h")
+
+_lib = None
+
+STATUS = {0: "NVQ_OK", 1: "NVQ_ERR_INVALID_ARG", 2: "NVQ_ERR_UNSUPPORTED_SHAPE", 3: "NVQ_ERR_MISALIGNED",
+          4: "NVQ_ERR_WORKSPACE", 5: "NVQ_ERR_CUDA", 6: "NVQ_ERR_DEVICE_TIMEOUT"}
+
+
+class NvqError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} {detail}".rstrip())
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/nvq.h."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+([a-z][a-z0-9_]*)\s*\(", text, flags=re.M)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libnvq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libnvq.so not built at {LIB_PATH}; run "
+                               "`python -m phase_disaggregated_quantized_b200.build_lib`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, sz, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+        sig = {
+            "nvq_abi_version": ([], i32),
+            "nvq_status_string": ([i32], ctypes.c_char_p),
+            "nvq_last_error_detail": ([], ctypes.c_char_p),
+            "nvq_check_device_error": ([vp], i32),
+            "nvfp4_scales_bytes": ([i64, i64], sz),
+            "nvfp4_quantize_workspace_bytes": ([i64, i64], sz),
+            "nvfp4_quantize": ([vp, i64, i64, vp, vp, vp, vp, vp, sz, vp], i32),
+            "nvfp4_gemm_w4a4": ([vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
+            "int4_quantize": ([vp, i64, i64, vp, vp, vp], i32),
+            "int4_pack_weights": ([vp, vp, i64, i64, vp, vp, vp], i32),
+            "w4a16_workspace_bytes": ([i64, i64, i64], sz),
+            "w4a16_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp, sz, vp], i32),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes, fn.restype = args, res
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise NvqError(status, where, lib().nvq_last_error_detail().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libnvq calls take CUDA tensors")
+
+
+def nvfp4_scales_bytes(rows: int, K: int) -> int:
+    return int(lib().nvfp4_scales_bytes(rows, K))
+
+
+def nvfp4_quantize_workspace_bytes(rows: int, K: int) -> int:
+    return int(lib().nvfp4_quantize_workspace_bytes(rows, K))
+
+
+def w4a16_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().w4a16_workspace_bytes(M, N, K))
+
+
+def check_device_error(stream=None):
+    _check(lib().nvq_check_device_error(_stream(stream)), "nvq_check_device_error")
+
+
+def nvfp4_quantize(x, tensor_scale_in=None, *, codes=None, scales=None, tensor_scale_out=None, workspace=None,
+                   stream=None):
+    """BF16 [rows, K] -> (codes uint8 [rows, K/2], tiled scales uint8, t float32 [1])."""
+    _need_cuda(x, tensor_scale_in)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+    rows, K = x.shape
+    dev = x.device
+    if codes is None:
+        codes = torch.empty(rows, K // 2, dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(max(1, nvfp4_scales_bytes(rows, K)), dtype=torch.uint8, device=dev)
+    if tensor_scale_out is None:
+        tensor_scale_out = torch.empty(1, dtype=torch.float32, device=dev)
+    need = nvfp4_quantize_workspace_bytes(rows, K) if tensor_scale_in is None else 0
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().nvfp4_quantize(_ptr(x), rows, K, _ptr(tensor_scale_in), _ptr(codes), _ptr(scales),
+                                _ptr(tensor_scale_out), _ptr(workspace), ws_bytes, _stream(stream)),
+           "nvfp4_quantize")
+    return codes, scales, tensor_scale_out
+
+
+def nvfp4_gemm_w4a4(xq, wq, M: int, N: int, K: int, *, y=None, stream=None):
+    """Y [M, N] bf16 = dequant(xq) @ dequant(wq)^T; xq / wq are (codes, scales, t)."""
+    xc, xs, tx = xq
+    wc, ws, tw = wq
+    _need_cuda(xc, xs, tx, wc, ws, tw)
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=xc.device)
+    _check(lib().nvfp4_gemm_w4a4(_ptr(xc), _ptr(xs), _ptr(tx), _ptr(wc), _ptr(ws), _ptr(tw), _ptr(y), M, N, K,
+                                 _stream(stream)), "nvfp4_gemm_w4a4")
+    return y
+
+
+def int4_quantize(w, *, codes=None, scales=None, stream=None):
+    """BF16 [N, K] -> (codes uint8 [N, K/2], scales bf16 [N, K/128])."""
+    _need_cuda(w)
+    assert w.dtype == torch.bfloat16 and w.dim() == 2 and w.is_contiguous()
+    N, K = w.shape
+    if codes is None:
+        codes = torch.empty(N, K // 2, dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty(N, K // 128, dtype=torch.bfloat16, device=w.device)
+    _check(lib().int4_quantize(_ptr(w), N, K, _ptr(codes), _ptr(scales), _stream(stream)), "int4_quantize")
+    return codes, scales
+
+
+def int4_pack_weights(codes, scales, N: int, K: int, *, packed_codes=None, packed_scales=None, stream=None):
+    """Offline reorder into the decode kernel's fragment order."""
+    _need_cuda(codes, scales)
+    if packed_codes is None:
+        packed_codes = torch.empty(N * K // 2, dtype=torch.uint8, device=codes.device)
+    if packed_scales is None:
+        packed_scales = torch.empty(N * (K // 128) * 2, dtype=torch.uint8, device=codes.device)
+    _check(lib().int4_pack_weights(_ptr(codes), _ptr(scales), N, K, _ptr(packed_codes), _ptr(packed_scales),
+                                   _stream(stream)), "int4_pack_weights")
+    return packed_codes, packed_scales
+
+
+def w4a16_gemm(x, packed_codes, packed_scales, N: int, *, y=None, workspace=None, stream=None):
+    """BF16 X [M, K] times packed INT4 W [N, K] -> Y [M, N] bf16."""
+    _need_cuda(x, packed_codes, packed_scales)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+    M, K = x.shape
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    need = w4a16_workspace_bytes(M, N, K)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().w4a16_gemm(_ptr(x), _ptr(packed_codes), _ptr(packed_scales), _ptr(y), M, N, K, _ptr(workspace),
+                            ws_bytes, _stream(stream)), "w4a16_gemm")
+    return y

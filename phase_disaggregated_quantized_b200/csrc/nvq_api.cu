@@ -1,0 +1,326 @@
+// Host side of the libnvq C ABI (include/nvq.h): argument validation, TMA
+// descriptor encoding and kernel launches.  All kernels live in this single
+// translation unit so the device error word needs no relocatable device code.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/nvq.h"
+#include "int4.cuh"
+#include "nvfp4_gemm.cuh"
+#include "nvfp4_quantize.cuh"
+#include "ptx.cuh"
+#include "w4a16_gemm.cuh"
+
+namespace {
+
+thread_local char g_detail[256] = "";
+
+nvq_status cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_detail, sizeof(g_detail), "%s: %s", where, cudaGetErrorString(e));
+  return NVQ_ERR_CUDA;
+}
+
+nvq_status fail(nvq_status s, const char* what) {
+  snprintf(g_detail, sizeof(g_detail), "%s", what);
+  return s;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+nvq_status launch_status(const char* where) {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? NVQ_OK : cuda_fail(e, where);
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor map: inner dimension `inner` elements, `outer` rows,
+// row pitch `pitch_bytes`, box {box_inner, box_outer}, 128-byte swizzle.
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                 uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int64_t kMaxDim = (int64_t)1 << 31;
+
+// Decode split of K: enough warps to cover the SMs, only at small batch.
+uint32_t w4a16_splits(int64_t M, int64_t N, int64_t K) {
+  const uint32_t G = (uint32_t)(K / 128);
+  if (M > 64) return 1;
+  const uint64_t tiles = (uint64_t)(N / 16);
+  uint32_t best = 1;
+  for (uint32_t s = 1; s <= G; ++s) {
+    if (G % s) continue;
+    best = s;
+    if (tiles * s >= 2048) break;
+  }
+  return best;
+}
+
+template <int NT8>
+nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* y, float* ws, int64_t M,
+                               int64_t N, int64_t K, uint32_t splits, cudaStream_t stream) {
+  using namespace nvq::w4a16;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(w4a16_kernel<NT8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem_bytes<NT8>());
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "w4a16_gemm: smem attribute");
+  const uint32_t G = (uint32_t)(K / 128);
+  const uint32_t gps = G / splits;
+  const uint32_t cta_rows = (uint32_t)((N / 16 + WARPS - 1) / WARPS);
+  const uint64_t grid = (uint64_t)cta_rows * splits;
+  w4a16_kernel<NT8><<<(unsigned)grid, THREADS, smem_bytes<NT8>(), stream>>>(
+      static_cast<const __nv_bfloat16*>(x), reinterpret_cast<const uint4*>(pc), static_cast<const uint32_t*>(ps),
+      static_cast<__nv_bfloat16*>(y), ws, (uint32_t)M, (uint32_t)N, (uint32_t)K, gps, splits);
+  return launch_status("w4a16_kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+int nvq_abi_version(void) { return 1; }
+
+const char* nvq_status_string(nvq_status s) {
+  switch (s) {
+    case NVQ_OK: return "NVQ_OK";
+    case NVQ_ERR_INVALID_ARG: return "NVQ_ERR_INVALID_ARG";
+    case NVQ_ERR_UNSUPPORTED_SHAPE: return "NVQ_ERR_UNSUPPORTED_SHAPE";
+    case NVQ_ERR_MISALIGNED: return "NVQ_ERR_MISALIGNED";
+    case NVQ_ERR_WORKSPACE: return "NVQ_ERR_WORKSPACE";
+    case NVQ_ERR_CUDA: return "NVQ_ERR_CUDA";
+    case NVQ_ERR_DEVICE_TIMEOUT: return "NVQ_ERR_DEVICE_TIMEOUT";
+  }
+  return "NVQ_ERR_UNKNOWN";
+}
+
+const char* nvq_last_error_detail(void) { return g_detail; }
+
+nvq_status nvq_check_device_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "nvq_check_device_error: synchronize");
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, nvq::g_device_error, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "nvq_check_device_error: read");
+  if (word != 0u) {
+    const unsigned int zero = 0u;
+    e = cudaMemcpyToSymbol(nvq::g_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "nvq_check_device_error: clear");
+    return fail(NVQ_ERR_DEVICE_TIMEOUT, "a kernel gave up on a bounded wait");
+  }
+  return NVQ_OK;
+}
+
+// ------------------------------------------------------------------ NVFP4 quantize
+size_t nvfp4_scales_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K <= 0 || K % 64) return 0;
+  return (size_t)((rows + 127) / 128 * 128) * (size_t)(K / 16);
+}
+
+size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K) {
+  if (rows <= 0 || K <= 0) return 0;
+  return (size_t)nvq::kAmaxMaxBlocks * sizeof(float);
+}
+
+nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const float* tensor_scale_in,
+                          uint8_t* codes, uint8_t* scales, float* tensor_scale_out, void* workspace,
+                          size_t workspace_bytes, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (rows < 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_quantize: rows < 0 or K <= 0");
+  if (K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize: K % 64 != 0");
+  if (rows >= kMaxDim || K >= kMaxDim || (rows * (K / 16)) >= ((int64_t)1 << 40))
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize: tensor too large");
+  if (tensor_scale_out == nullptr) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_quantize: tensor_scale_out is NULL");
+  if (rows > 0 && (x_bf16 == nullptr || codes == nullptr || scales == nullptr))
+    return fail(NVQ_ERR_INVALID_ARG, "nvfp4_quantize: NULL tensor pointer");
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales))
+    return fail(NVQ_ERR_MISALIGNED, "nvfp4_quantize: pointer not 16-byte aligned");
+  const bool need_amax = tensor_scale_in == nullptr && rows > 0;
+  int amax_blocks = 0;
+  if (need_amax) {
+    const size_t nvec = (size_t)rows * (size_t)K / 8;
+    amax_blocks = (int)std::min<size_t>(nvq::kAmaxMaxBlocks, (nvec + 4 * nvq::kAmaxThreads - 1) /
+                                                                 (4 * nvq::kAmaxThreads));
+    if (amax_blocks < 1) amax_blocks = 1;
+    if (workspace == nullptr || workspace_bytes < (size_t)amax_blocks * sizeof(float))
+      return fail(NVQ_ERR_WORKSPACE, "nvfp4_quantize: workspace missing or too small");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
+      return fail(NVQ_ERR_MISALIGNED, "nvfp4_quantize: workspace not 4-byte aligned");
+    nvq::nvfp4_amax_kernel<<<amax_blocks, nvq::kAmaxThreads, 0, stream>>>(
+        static_cast<const uint4*>(x_bf16), nvec, static_cast<float*>(workspace));
+    nvq_status st = launch_status("nvfp4_amax_kernel");
+    if (st != NVQ_OK) return st;
+  }
+  const uint64_t nblocks = (uint64_t)rows * (uint64_t)(K / 16);
+  const uint64_t want = (nblocks + nvq::kQuantThreads - 1) / nvq::kQuantThreads;
+  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count() * 8));
+  nvq::nvfp4_quantize_kernel<<<grid, nvq::kQuantThreads, 0, stream>>>(
+      static_cast<const uint4*>(x_bf16), (uint32_t)rows, (uint32_t)K, tensor_scale_in,
+      static_cast<const float*>(workspace), amax_blocks, reinterpret_cast<uint2*>(codes), scales,
+      tensor_scale_out);
+  return launch_status("nvfp4_quantize_kernel");
+}
+
+// ------------------------------------------------------------------ NVFP4 GEMM
+nvq_status nvfp4_gemm_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const float* t_x,
+                           const uint8_t* w_codes, const uint8_t* w_scales, const float* t_w, void* y_bf16,
+                           int64_t M, int64_t N, int64_t K, void* stream_) {
+  using namespace nvq::w4a4;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4: bad sizes");
+  if (N % 8 != 0 || K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4: need N % 8 == 0, K % 64 == 0");
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4: too large");
+  if (!x_codes || !x_scales || !t_x || !w_codes || !w_scales || !t_w || !y_bf16)
+    return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4: NULL pointer");
+  if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(y_bf16) || (reinterpret_cast<uintptr_t>(t_x) & 3u) || (reinterpret_cast<uintptr_t>(t_w) & 3u))
+    return fail(NVQ_ERR_MISALIGNED, "nvfp4_gemm_w4a4: pointer not aligned");
+  if (M == 0) return NVQ_OK;
+  CUtensorMap ma, mb, my;
+  if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
+                   BKB, BM) ||
+      !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
+                   BKB, BN) ||
+      !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2,
+                   C_CHUNK_COLS, BM))
+    return fail(NVQ_ERR_CUDA, "nvfp4_gemm_w4a4: tensor map encoding failed");
+  Params p;
+  p.x_scales = x_scales;
+  p.w_scales = w_scales;
+  p.t_x = t_x;
+  p.t_w = t_w;
+  p.M = (uint32_t)M;
+  p.N = (uint32_t)N;
+  p.K = (uint32_t)K;
+  p.num_m_tiles = (uint32_t)((M + BM - 1) / BM);
+  p.num_n_tiles = (uint32_t)((N + BN - 1) / BN);
+  p.num_k_stages = (uint32_t)((K / 2 + BKB - 1) / BKB);
+  p.k_atoms = (uint32_t)(K / 64);
+  p.n_row_atoms = (uint32_t)((N + 127) / 128);
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "nvfp4_gemm_w4a4: smem attribute");
+  const uint64_t tiles = (uint64_t)p.num_m_tiles * p.num_n_tiles;
+  const int grid = (int)std::min<uint64_t>(tiles, (uint64_t)sm_count());
+  nvfp4_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, my, p);
+  return launch_status("nvfp4_gemm_kernel");
+}
+
+// ------------------------------------------------------------------ INT4
+nvq_status int4_quantize(const void* w_bf16, int64_t N, int64_t K, uint8_t* codes, void* scales_bf16,
+                         void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (N < 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "int4_quantize: bad sizes");
+  if (K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_quantize: K % 128 != 0");
+  if (N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_quantize: too large");
+  if (N == 0) return NVQ_OK;
+  if (!w_bf16 || !codes || !scales_bf16) return fail(NVQ_ERR_INVALID_ARG, "int4_quantize: NULL pointer");
+  if (!aligned16(w_bf16) || !aligned16(codes) || !aligned16(scales_bf16))
+    return fail(NVQ_ERR_MISALIGNED, "int4_quantize: pointer not 16-byte aligned");
+  const uint64_t groups = (uint64_t)N * (uint64_t)(K / 128);
+  const uint64_t want = (groups + 7) / 8;
+  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count() * 16));
+  nvq::int4_quantize_kernel<<<grid, nvq::kInt4QuantThreads, 0, stream>>>(
+      static_cast<const uint2*>(w_bf16), (uint32_t)N, (uint32_t)K, reinterpret_cast<uint16_t*>(codes),
+      static_cast<uint16_t*>(scales_bf16));
+  return launch_status("int4_quantize_kernel");
+}
+
+nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int64_t N, int64_t K,
+                             uint8_t* packed_codes, void* packed_scales, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (N < 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "int4_pack_weights: bad sizes");
+  if (N % 16 != 0 || K % 128 != 0)
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_pack_weights: need N % 16 == 0, K % 128 == 0");
+  if (N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_pack_weights: too large");
+  if (N == 0) return NVQ_OK;
+  if (!codes || !scales_bf16 || !packed_codes || !packed_scales)
+    return fail(NVQ_ERR_INVALID_ARG, "int4_pack_weights: NULL pointer");
+  if (!aligned16(codes) || !aligned16(scales_bf16) || !aligned16(packed_codes) || !aligned16(packed_scales))
+    return fail(NVQ_ERR_MISALIGNED, "int4_pack_weights: pointer not 16-byte aligned");
+  const uint64_t nwords = (uint64_t)N * (uint64_t)K / 8;
+  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>((nwords + 255) / 256, (uint64_t)sm_count() * 16));
+  nvq::int4_pack_kernel<<<grid, 256, 0, stream>>>(codes, static_cast<const uint16_t*>(scales_bf16), (uint32_t)N,
+                                                  (uint32_t)K, reinterpret_cast<uint32_t*>(packed_codes),
+                                                  static_cast<uint32_t*>(packed_scales));
+  return launch_status("int4_pack_kernel");
+}
+
+// ------------------------------------------------------------------ W4A16 decode GEMM
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0 || N % 16 || K % 128) return 0;
+  const uint32_t s = w4a16_splits(M, N, K);
+  return s <= 1 ? 0 : (size_t)s * (size_t)M * (size_t)N * sizeof(float);
+}
+
+nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const void* packed_scales, void* y_bf16,
+                      int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "w4a16_gemm: bad sizes");
+  if (N % 16 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_gemm: need N % 16 == 0, K % 128 == 0");
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_gemm: too large");
+  if (M == 0) return NVQ_OK;
+  if (!x_bf16 || !packed_codes || !packed_scales || !y_bf16) return fail(NVQ_ERR_INVALID_ARG, "w4a16_gemm: NULL pointer");
+  if (!aligned16(x_bf16) || !aligned16(packed_codes) || !aligned16(packed_scales) || !aligned16(y_bf16))
+    return fail(NVQ_ERR_MISALIGNED, "w4a16_gemm: pointer not 16-byte aligned");
+  const uint32_t splits = w4a16_splits(M, N, K);
+  float* ws = nullptr;
+  if (splits > 1) {
+    const size_t need = (size_t)splits * (size_t)M * (size_t)N * sizeof(float);
+    if (workspace == nullptr || workspace_bytes < need) return fail(NVQ_ERR_WORKSPACE, "w4a16_gemm: workspace too small");
+    if (!aligned16(workspace)) return fail(NVQ_ERR_MISALIGNED, "w4a16_gemm: workspace not 16-byte aligned");
+    ws = static_cast<float*>(workspace);
+  }
+  nvq_status st;
+  if (M <= 8) st = launch_w4a16<1>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, splits, stream);
+  else if (M <= 16) st = launch_w4a16<2>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, splits, stream);
+  else st = launch_w4a16<4>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, splits, stream);
+  if (st != NVQ_OK || splits == 1) return st;
+  const uint64_t n4 = (uint64_t)M * (uint64_t)N / 4;
+  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>((n4 + 255) / 256, (uint64_t)sm_count() * 8));
+  nvq::w4a16::w4a16_reduce_kernel<<<grid, 256, 0, stream>>>(static_cast<const float4*>(workspace),
+                                                            static_cast<uint2*>(y_bf16), splits, n4);
+  return launch_status("w4a16_reduce_kernel");
+}
+
+}  // extern "C"

@@ -1,0 +1,108 @@
+"""The C-ABI library: loads without a GPU, exports every declared entry point,
+and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+
+import pytest
+
+import phase_disaggregated_quantized_b200 as nvq
+from phase_disaggregated_quantized_b200 import build_lib
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_lib.build()
+    return nvq.lib()
+
+
+def test_header_lists_the_entry_points():
+    names = nvq.header_functions()
+    for must in ("nvfp4_quantize", "nvfp4_gemm_w4a4", "int4_pack_weights", "w4a16_gemm", "int4_quantize",
+                 "nvq_check_device_error", "nvfp4_scales_bytes", "w4a16_workspace_bytes"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in nvq.header_functions():
+        assert hasattr(L, name), name
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.nvq_abi_version() == 1
+    for code, name in nvq.STATUS.items():
+        assert L.nvq_status_string(code).decode() == name
+
+
+def test_size_helpers(L):
+    assert L.nvfp4_scales_bytes(1, 64) == 128 * 4
+    assert L.nvfp4_scales_bytes(130, 512) == 256 * 32
+    assert L.nvfp4_scales_bytes(10, 100) == 0          # K % 64 != 0
+    assert L.nvfp4_quantize_workspace_bytes(0, 64) == 0
+    assert L.nvfp4_quantize_workspace_bytes(128, 512) > 0
+    assert L.w4a16_workspace_bytes(1, 4096, 4096) % 4 == 0
+    assert L.w4a16_workspace_bytes(4096, 4096, 4096) == 0   # no split at large batch
+
+
+FAKE = 0x7F0000000000          # 16-byte aligned, never dereferenced: validation fails first
+ODD = FAKE + 8
+
+
+def _vp(v):
+    return ctypes.c_void_p(v)
+
+
+def test_quantize_rejects_bad_arguments(L):
+    q = L.nvfp4_quantize
+    assert q(_vp(FAKE), 4, 100, None, _vp(FAKE), _vp(FAKE), _vp(FAKE), None, 0, None) == 2   # K % 64
+    assert q(_vp(FAKE), -1, 64, None, _vp(FAKE), _vp(FAKE), _vp(FAKE), None, 0, None) == 1
+    assert q(_vp(FAKE), 4, 64, None, _vp(FAKE), _vp(FAKE), None, None, 0, None) == 1          # no t_out
+    assert q(_vp(ODD), 4, 64, None, _vp(FAKE), _vp(FAKE), _vp(FAKE), None, 0, None) == 3
+    assert q(_vp(FAKE), 4, 64, None, _vp(FAKE), _vp(FAKE), _vp(FAKE), None, 0, None) == 4     # workspace
+    assert q(_vp(FAKE), 4, 64, None, _vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 2, None) == 4
+    assert b"workspace" in L.nvq_last_error_detail()
+
+
+def test_gemm_rejects_bad_arguments(L):
+    g = L.nvfp4_gemm_w4a4
+    a = [_vp(FAKE)] * 7
+    assert g(*a, 128, 12, 512, None) == 2            # N % 8
+    assert g(*a, 128, 512, 96, None) == 2            # K % 64
+    assert g(*a, -1, 512, 512, None) == 1
+    b = list(a)
+    b[6] = _vp(ODD)
+    assert g(*b, 128, 512, 512, None) == 3
+    b = list(a)
+    b[0] = None
+    assert g(*b, 128, 512, 512, None) == 1
+
+
+def test_int4_calls_reject_bad_arguments(L):
+    assert L.int4_quantize(_vp(FAKE), 16, 100, _vp(FAKE), _vp(FAKE), None) == 2
+    assert L.int4_pack_weights(_vp(FAKE), _vp(FAKE), 24, 128, _vp(FAKE), _vp(FAKE), None) == 2   # N % 16
+    assert L.int4_pack_weights(_vp(ODD), _vp(FAKE), 32, 128, _vp(FAKE), _vp(FAKE), None) == 3
+    w = L.w4a16_gemm
+    assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 24, 128, None, 0, None) == 2
+    assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 4096, 4096, None, 0, None) == 4   # split-K workspace
+    assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(ODD), 4, 4096, 4096, _vp(FAKE), 1 << 30, None) == 3
+
+
+def test_zero_sized_calls_are_noops(L):
+    assert L.nvfp4_gemm_w4a4(*([_vp(FAKE)] * 7), 0, 512, 512, None) == 0
+    assert L.w4a16_gemm(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 0, 512, 512, None, 0, None) == 0
+    assert L.int4_quantize(_vp(FAKE), 0, 128, _vp(FAKE), _vp(FAKE), None) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(nvq, "LIB_PATH", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(nvq, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        nvq.lib()
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.dirname(nvq.__file__)
+    for root, _dirs, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(root, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f

@@ -1,0 +1,309 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the CPU oracle.
+
+Bar: quantized codes, block scales and tensor scales bit-exact; GEMM outputs
+within |y - y_ref| <= 8e-3 |y_ref| + 1e-3 rms(y_ref).  Inputs come from the
+seeded generators (phase_disaggregated_quantized_b200.synth) or are built here
+on and around the rounding decision points.
+"""
+import numpy as np
+import pytest
+import torch
+
+import phase_disaggregated_quantized_b200 as nvq
+from phase_disaggregated_quantized_b200 import synth
+from oracle import int4 as oint4
+from oracle import nvfp4 as onv
+
+from helpers import bf16_bits, bf16_to_f64, oracle_int4, oracle_nvfp4, u8
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    from phase_disaggregated_quantized_b200 import build_lib
+    build_lib.build()
+    nvq.lib()
+    yield
+    nvq.check_device_error()
+
+
+def gpu_quant(x_cpu, t_in=None):
+    x = x_cpu.cuda()
+    tin = None if t_in is None else torch.tensor([t_in], dtype=torch.float32, device="cuda")
+    c, s, t = nvq.nvfp4_quantize(x, tin)
+    nvq.check_device_error()
+    return c, s, t
+
+
+def assert_quant_parity(x_cpu, t_in=None):
+    rows, K = x_cpu.shape
+    pc, s, t = oracle_nvfp4(x_cpu, t_in)
+    gc, gs, gt = gpu_quant(x_cpu, t_in)
+    assert float(gt.item()) == t
+    np.testing.assert_array_equal(u8(gc), pc)
+    np.testing.assert_array_equal(u8(gs), onv.scales_to_tiled(s, rows, K))   # padding rows zero too
+    return gc, gs, gt
+
+
+def _bf16_tensor(values) -> torch.Tensor:
+    return torch.tensor(np.asarray(values, dtype=np.float32)).to(torch.bfloat16)
+
+
+# ------------------------------------------------------------------ NVFP4 quantize
+
+def test_quantize_tiny_case_bit_exact():
+    x, w = synth.tiny_case()
+    assert_quant_parity(x)
+    assert_quant_parity(w)
+
+
+@pytest.mark.parametrize("rows,K", [(1, 64), (77, 192), (130, 1024), (300, 512), (129, 4096)])
+def test_quantize_ragged_shapes(rows, K):
+    assert_quant_parity(synth.activations(rows, K, seed=rows * 7 + K))
+
+
+def test_quantize_caller_scale_and_saturation():
+    x = synth.activations(64, 256, seed=3)
+    assert_quant_parity(x, t_in=0.01)
+    assert_quant_parity(x, t_in=1e-6)        # every block scale clamps at 448
+    assert_quant_parity(x, t_in=3.0)         # many blocks underflow to a zero scale
+
+
+def test_quantize_zero_and_signed_zero():
+    x = torch.zeros(130, 128, dtype=torch.bfloat16)
+    x[5, 7] = -0.0
+    x[129, 127] = -0.0
+    gc, gs, gt = assert_quant_parity(x)
+    assert float(gt.item()) == 1.0
+
+
+def _decision_point_tensor(seed, t, rows=64, K=512):
+    """Elements on and one bf16 ulp around mu_i * S * t for random E4M3 scales S."""
+    g = np.random.default_rng(seed)
+    out = np.zeros((rows, K), dtype=np.float32)
+    mids = onv.E2M1_MIDPOINTS
+    for r in range(rows):
+        for b in range(K // 16):
+            S = onv.e4m3_value(int(g.integers(1, 127)))
+            d = S * t
+            vals = [6 * d] + [float(g.choice(mids)) * d for _ in range(15)]
+            out[r, 16 * b:16 * b + 16] = vals
+    xb = torch.tensor(out).to(torch.bfloat16)
+    bits = xb.view(torch.int16)
+    bits += torch.tensor(g.integers(-1, 2, size=(rows, K)), dtype=torch.int16)
+    xb = bits.view(torch.bfloat16)
+    sign = torch.tensor(g.integers(0, 2, size=(rows, K)).astype(bool))
+    xb[sign] = -xb[sign]
+    return xb
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_quantize_decision_points_bit_exact(seed):
+    t = float(np.float32(1.3 ** (seed - 2) / 2688 * 17.0))
+    x = _decision_point_tensor(seed, t)
+    assert_quant_parity(x, t_in=t)           # ties and near-ties under a caller scale
+    assert_quant_parity(x)                   # and under the computed scale
+
+
+def test_quantize_grid_round_trip():
+    g = np.random.default_rng(4)
+    rows, K = 8, 256
+    vals = np.zeros((rows, K))
+    vals[0, 0] = 2688.0
+    for r in range(rows):
+        for b in range(K // 16):
+            if r == 0 and b == 0:
+                continue
+            S = onv.e4m3_value(int(g.integers(1, 100)))
+            c = g.integers(0, 8, size=16)
+            c[g.integers(16)] = 7
+            vals[r, 16 * b:16 * b + 16] = onv.E2M1_MAGNITUDES[c] * S * np.where(g.random(16) < 0.5, -1, 1)
+    x = _bf16_tensor(vals)
+    gc, gs, gt = assert_quant_parity(x)
+    assert float(gt.item()) == 1.0
+    deq = onv.dequantize(onv.unpack_codes(u8(gc)), onv.scales_from_tiled(u8(gs), rows, K), 1.0)
+    np.testing.assert_array_equal(deq, bf16_to_f64(x))
+
+
+# ------------------------------------------------------------------ NVFP4 GEMM
+
+def gemm_case(x_cpu, w_cpu, t_in_x=None, t_in_w=None):
+    M, K = x_cpu.shape
+    N = w_cpu.shape[0]
+    xq = gpu_quant(x_cpu, t_in_x)
+    wq = gpu_quant(w_cpu, t_in_w)
+    y = nvq.nvfp4_gemm_w4a4(xq, wq, M, N, K)
+    nvq.check_device_error()
+    xc, xs, tx = onv.quantize(bf16_to_f64(x_cpu), t_in=t_in_x)
+    wc, ws, tw = onv.quantize(bf16_to_f64(w_cpu), t_in=t_in_w)
+    y_ref = onv.gemm_ref(onv.dequantize(xc, xs, tx), onv.dequantize(wc, ws, tw))
+    return bf16_to_f64(y), y_ref
+
+
+def test_gemm_tiny_case():
+    x, w = synth.tiny_case()
+    y, y_ref = gemm_case(x, w)
+    ok, worst = onv.within_tolerance(y, y_ref)
+    assert ok, worst
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 64), (77, 136, 192), (200, 264, 320), (129, 520, 1024),
+                                   (300, 256, 4096), (256, 512, 256), (5, 1000, 128)])
+def test_gemm_ragged_shapes(M, N, K):
+    x = synth.activations(M, K, seed=M + N + K)
+    w = synth.weights(N, K, seed=M * N)
+    y, y_ref = gemm_case(x, w)
+    ok, worst = onv.within_tolerance(y, y_ref)
+    assert ok, (M, N, K, worst)
+
+
+def test_gemm_unit_scales_exact_integer_case():
+    """All block scales 1 and t = 1: Y = RNE_bf16 of an exact quarter-integer sum."""
+    g = np.random.default_rng(8)
+    M, N, K = 200, 264, 512
+    cx = g.integers(0, 16, size=(M, K))
+    cw = g.integers(0, 16, size=(N, K))
+    cx[:, ::16] = 7
+    cw[:, ::16] = 7 | 8
+    x = _bf16_tensor(onv.e2m1_signed(cx.astype(np.uint8)))
+    w = _bf16_tensor(onv.e2m1_signed(cw.astype(np.uint8)))
+    y, y_ref = gemm_case(x, w, 1.0, 1.0)
+    want = torch.tensor(y_ref, dtype=torch.float64).to(torch.float32).to(torch.bfloat16)
+    np.testing.assert_array_equal(y, bf16_to_f64(want))
+
+
+@pytest.mark.parametrize("layer", range(4))
+def test_gemm_qwen3_8b_prefill_full_size_sampled(layer):
+    """M = 8192 on each Qwen3-8B linear; sampled rows and columns against the oracle."""
+    name, K, N = synth.QWEN3_8B_LINEARS[layer]
+    M = 8192
+    x = synth.activations(M, K, seed=2000 + 10 * layer)
+    w = synth.weights(N, K, seed=2000 + 10 * layer)
+    gx = gpu_quant(x)
+    gw = gpu_quant(w)
+    y = nvq.nvfp4_gemm_w4a4(gx, gw, M, N, K)
+    nvq.check_device_error()
+    g = np.random.default_rng(layer)
+    mi = np.sort(g.choice(M, 48, replace=False))
+    ni = np.sort(g.choice(N, 48, replace=False))
+    xf, wf = bf16_to_f64(x), bf16_to_f64(w)
+    tx, tw = onv.tensor_scale(xf), onv.tensor_scale(wf)
+    xc, xs, _ = onv.quantize(xf[mi], t_in=tx)
+    wc, ws, _ = onv.quantize(wf[ni], t_in=tw)
+    assert float(gx[2].item()) == tx and float(gw[2].item()) == tw
+    # codes and scales of the sampled rows, bit-exact
+    np.testing.assert_array_equal(u8(gx[0])[mi], onv.pack_codes(xc))
+    np.testing.assert_array_equal(onv.scales_from_tiled(u8(gx[1]), M, K)[mi], xs)
+    np.testing.assert_array_equal(onv.scales_from_tiled(u8(gw[1]), N, K)[ni], ws)
+    y_ref = onv.gemm_ref(onv.dequantize(xc, xs, tx), onv.dequantize(wc, ws, tw))
+    y_s = bf16_to_f64(y[torch.tensor(mi).cuda()][:, torch.tensor(ni).cuda()])
+    ok, worst = onv.within_tolerance(y_s, y_ref)
+    assert ok, (name, worst)
+
+
+# ------------------------------------------------------------------ INT4 / W4A16
+
+def gpu_int4(w_cpu):
+    N, K = w_cpu.shape
+    codes, scales = nvq.int4_quantize(w_cpu.cuda())
+    pc, ps = nvq.int4_pack_weights(codes, scales, N, K)
+    nvq.check_device_error()
+    return codes, scales, pc, ps
+
+
+@pytest.mark.parametrize("N,K", [(512, 512), (16, 128), (4096, 4096), (48, 384)])
+def test_int4_quantize_and_pack_bit_exact(N, K):
+    w = synth.weights(N, K, seed=N + K)
+    if N == 48:
+        w[3, :128] = 0                                       # an all-zero group
+    codes, scales, pc, ps = gpu_int4(w)
+    u, s_bits = oracle_int4(w)
+    np.testing.assert_array_equal(u8(codes), oint4.pack_nibbles(u))
+    np.testing.assert_array_equal(bf16_bits(scales), s_bits)
+    opc, ops = oint4.pack_weights(u, s_bits)
+    np.testing.assert_array_equal(u8(pc), opc)
+    np.testing.assert_array_equal(u8(ps), ops)
+    u2, s2 = oint4.unpack_weights(u8(pc), u8(ps), N, K)
+    np.testing.assert_array_equal(u2, u)
+    np.testing.assert_array_equal(s2, s_bits)
+
+
+def w4a16_case(x_cpu, w_cpu, packed=None):
+    N, K = w_cpu.shape
+    if packed is None:
+        packed = gpu_int4(w_cpu)
+    _, _, pc, ps = packed
+    y = nvq.w4a16_gemm(x_cpu.cuda(), pc, ps, N)
+    nvq.check_device_error()
+    u, s_bits = oracle_int4(w_cpu)
+    y_ref = oint4.w4a16_ref(bf16_to_f64(x_cpu), oint4.dequantize(u, s_bits))
+    return bf16_to_f64(y), y_ref
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_w4a16_tiny_case(M):
+    _, w = synth.tiny_case()
+    x = synth.activations(M, 512, seed=M, n_outliers=4)
+    y, y_ref = w4a16_case(x, w)
+    ok, worst = onv.within_tolerance(y, y_ref)
+    assert ok, worst
+
+
+@pytest.mark.parametrize("M,N,K", [(3, 1024, 1024), (13, 272, 384), (33, 1024, 2048), (100, 528, 640),
+                                   (1, 16, 128), (8, 8192, 128), (64, 4096, 1024)])
+def test_w4a16_ragged(M, N, K):
+    x = synth.activations(M, K, seed=M + K)
+    w = synth.weights(N, K, seed=N)
+    y, y_ref = w4a16_case(x, w)
+    ok, worst = onv.within_tolerance(y, y_ref)
+    assert ok, (M, N, K, worst)
+
+
+@pytest.mark.parametrize("layer", range(4))
+def test_w4a16_qwen3_8b_decode_full_size(layer):
+    name, K, N = synth.QWEN3_8B_LINEARS[layer]
+    w = synth.weights(N, K, seed=3000 + 10 * layer)
+    packed = gpu_int4(w)
+    for M in synth.DECODE_BATCHES:
+        x = synth.activations(M, K, seed=3000 + 10 * layer + M)
+        y, y_ref = w4a16_case(x, w, packed)
+        ok, worst = onv.within_tolerance(y, y_ref)
+        assert ok, (name, M, worst)
+
+
+@pytest.mark.parametrize("M", synth.CROSSOVER_BATCHES)
+def test_crossover_sweep_both_paths_sampled(M):
+    """gate_up (K=4096, N=24576): one master W quantized both ways, both paths at M."""
+    K, N = 4096, 24576
+    w = synth.weights(N, K, seed=5000)
+    x = synth.activations(M, K, seed=5000 + M)
+    g = np.random.default_rng(M)
+    mi = np.sort(g.choice(M, min(M, 32), replace=False))
+    ni = np.sort(g.choice(N, 64, replace=False))
+    xf, wf = bf16_to_f64(x), bf16_to_f64(w)
+    # W4A4
+    gx, gw = gpu_quant(x), gpu_quant(w)
+    y4 = nvq.nvfp4_gemm_w4a4(gx, gw, M, N, K)
+    tx, tw = onv.tensor_scale(xf), onv.tensor_scale(wf)
+    xc, xs, _ = onv.quantize(xf[mi], t_in=tx)
+    wc, ws, _ = onv.quantize(wf[ni], t_in=tw)
+    y_ref = onv.gemm_ref(onv.dequantize(xc, xs, tx), onv.dequantize(wc, ws, tw))
+    y_s = bf16_to_f64(y4[torch.tensor(mi).cuda()][:, torch.tensor(ni).cuda()])
+    ok, worst = onv.within_tolerance(y_s, y_ref)
+    assert ok, ("w4a4", M, worst)
+    # W4A16
+    _, _, pc, ps = gpu_int4(w)
+    y16 = nvq.w4a16_gemm(x.cuda(), pc, ps, N)
+    nvq.check_device_error()
+    u, s_bits = oint4.quantize(wf[ni])
+    y_ref = oint4.w4a16_ref(xf[mi], oint4.dequantize(u, s_bits))
+    y_s = bf16_to_f64(y16[torch.tensor(mi).cuda()][:, torch.tensor(ni).cuda()])
+    ok, worst = onv.within_tolerance(y_s, y_ref)
+    assert ok, ("w4a16", M, worst)
+
+
+def test_device_error_word_is_clear_after_normal_runs():
+    nvq.check_device_error()
