@@ -139,9 +139,10 @@ nvq_status int4_quantize(const void* w_bf16, int64_t N, int64_t K, uint8_t* code
  * Unit = 16 weight rows x one 128-wide group: 1024 code bytes at unit index
  * (n/16)*(K/128) + k/128.  Inside a unit, 32-bit word 128h + 4lane + jj (h in
  * {0,1}, lane = 4g + c in [0,32), jj in [0,4)) holds k16-step j = 4h + jj with
- * nibble p (bits 4p..4p+3) at (row, k-in-group):
- *   p=0 (g, 16j+2c)   p=4 (g, 16j+2c+1)   p=1 (g+8, 16j+2c)   p=5 (g+8, 16j+2c+1)
- *   p=2 (g, 16j+2c+8) p=6 (g, 16j+2c+9)   p=3 (g+8, 16j+2c+8) p=7 (g+8, 16j+2c+9)
+ * nibble p (bits 4p..4p+3) at (row, k-in-group); K is permuted inside the group
+ * so that lane (g, c) covers k = 32c .. 32c+31:
+ *   p=0 (g, 32c+4j)   p=4 (g, 32c+4j+1)   p=1 (g+8, 32c+4j)   p=5 (g+8, 32c+4j+1)
+ *   p=2 (g, 32c+4j+2) p=6 (g, 32c+4j+3)   p=3 (g+8, 32c+4j+2) p=7 (g+8, 32c+4j+3)
  * Scales: 32 bytes per unit; 32-bit word g holds rows g (low) and g+8 (high).
  *
  * codes [N, K/2] (as written by int4_quantize), scales_bf16 [N, K/128]

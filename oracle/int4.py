@@ -120,17 +120,18 @@ def bytes_ratio_bf16_over_int4_g128(group: int = GROUP, scale_bytes: int = 2) ->
 # The unit is a tile of 16 weight rows x one 128-wide group: 1024 code bytes
 # and 32 scale bytes, stored at unit index (n // 16) * (K / 128) + k // 128.
 # Inside a unit, 256 little-endian 32-bit words, word (h, lane, jj) at index
-# 128 h + 4 lane + jj holds k16-step j = 4 h + jj for lane = 4 g + c:
+# 128 h + 4 lane + jj holds k16-step j = 4 h + jj for lane = 4 g + c.  K is
+# permuted inside the group so that lane (g, c) covers k = 32c .. 32c+31:
 #   nibble p (bits 4p..4p+3), with r = row in tile, kk = k within the group:
-#     p=0: (g,   16j+2c)    p=4: (g,   16j+2c+1)
-#     p=1: (g+8, 16j+2c)    p=5: (g+8, 16j+2c+1)
-#     p=2: (g,   16j+2c+8)  p=6: (g,   16j+2c+9)
-#     p=3: (g+8, 16j+2c+8)  p=7: (g+8, 16j+2c+9)
+#     p=0: (g,   32c+4j)    p=4: (g,   32c+4j+1)
+#     p=1: (g+8, 32c+4j)    p=5: (g+8, 32c+4j+1)
+#     p=2: (g,   32c+4j+2)  p=6: (g,   32c+4j+3)
+#     p=3: (g+8, 32c+4j+2)  p=7: (g+8, 32c+4j+3)
 # Scale word g (g = 0..7) of a unit holds rows g (low half) and g+8 (high half).
 # ---------------------------------------------------------------------------
 
 _NIBBLE_ROW = np.array([0, 8, 0, 8, 0, 8, 0, 8])     # row offset added to g
-_NIBBLE_K = np.array([0, 0, 8, 8, 1, 1, 9, 9])       # k offset added to 16j+2c
+_NIBBLE_K = np.array([0, 0, 2, 2, 1, 1, 3, 3])       # k offset added to 32c+4j
 
 
 def packed_code_index(N: int, K: int):
@@ -144,7 +145,7 @@ def packed_code_index(N: int, K: int):
     j = 4 * h + jj
     g, c = lane // 4, lane % 4
     r = g[:, None] + _NIBBLE_ROW[None, :]                          # [256, 8]
-    kk = (16 * j + 2 * c)[:, None] + _NIBBLE_K[None, :]            # [256, 8]
+    kk = (32 * c + 4 * j)[:, None] + _NIBBLE_K[None, :]            # [256, 8]
     unit = np.arange(units)
     nt, gi = unit // G, unit % G
     n_idx = (16 * nt)[:, None, None] + r[None]                     # [units, 256, 8]

@@ -76,7 +76,7 @@ __global__ void int4_pack_kernel(const uint8_t* __restrict__ codes, const uint16
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
       const uint32_t r = 16 * nt + g + ((p & 1) ? 8u : 0u);
-      const uint32_t k = 128 * gi + 16 * j + 2 * c + ((p & 2) ? 8u : 0u) + ((p & 4) ? 1u : 0u);
+      const uint32_t k = 128 * gi + 32 * c + 4 * j + ((p & 2) ? 2u : 0u) + ((p & 4) ? 1u : 0u);
       const uint32_t byte = codes[(size_t)r * half_k + (k >> 1)];
       out |= ((byte >> (4 * (k & 1))) & 0xFu) << (4 * p);
     }

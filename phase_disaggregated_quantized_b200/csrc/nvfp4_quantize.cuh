@@ -14,13 +14,15 @@
 //     within one code of the exact answer; the two neighbouring midpoints are
 //     then tested exactly with the sign of fma(-(6 mu), t, amax_b), an exact
 //     product minus an exact value rounded once.
-//   * codes: q = |x| * (1/(S t)) in fp32 is within 3.01 ulp (relative 2^-24)
-//     of the exact quotient, so cvt.rn.satfinite.e2m1x2 on q decides like the
-//     exact quotient unless some bf16 value lies within 4.03 fp32 ulps of a
-//     threshold mu_i S t.  For each E4M3 scale code the kernel precomputes
-//     (once per CTA) whether that can happen; blocks with such a scale take an
-//     exact path that compares |x| against mu_i S t through its rounded value
+//   * codes: for each of the 127 E4M3 scale codes S the kernel derives, once
+//     per CTA, the exact decision thresholds as bf16 values: the smallest bf16
+//     that lies above mu_i S t (or on it, when the tie goes up), found from
 //     h = fl(P t) and the exact residual e = fma(P, t, -h), P = mu_i S exact.
+//     The fast path (q = |x| * fl(1/fl(S t)), cvt.rn.satfinite.e2m1x2) is used
+//     for a scale code only if it gives the exact code on both sides of every
+//     threshold; both maps are monotone in |x|, so it is then exact for every
+//     bf16 input.  Other scale codes count thresholds with packed bf16x2
+//     compares, which is exact by construction.
 #pragma once
 #include "ptx.cuh"
 
@@ -75,9 +77,12 @@ __global__ void __launch_bounds__(kAmaxThreads) nvfp4_amax_kernel(const uint4* _
 }
 
 // Value of a non-negative E4M3 (FN) code 0..126: bias 7, 3 mantissa bits.
+// Subnormals (exponent field 0) are m * 2^-9 = (1 + m/8) 2^-6 - 2^-6, exact.
 __device__ __forceinline__ float e4m3_value(uint32_t c) {
   const uint32_t e = c >> 3, m = c & 7u;
-  return e == 0 ? __int2float_rn((int)m) * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+  const float nrm = __uint_as_float(((e + 120u) << 23) | (m << 20));
+  const float sub = __fadd_rn(__uint_as_float((121u << 23) | (m << 20)), -0.015625f);
+  return e == 0 ? sub : nrm;
 }
 
 __device__ __forceinline__ uint32_t e4m3_rn_satfinite(float v) {
@@ -102,8 +107,10 @@ __device__ __forceinline__ bool scale_passes(float amax, float mu, float t, uint
   return r > 0.f || (r == 0.f && (upper_code & 1u) == 0u);
 }
 
-__device__ __forceinline__ uint32_t block_scale_code(float amax, float t, float t6) {
-  uint32_t s = e4m3_rn_satfinite(__fdiv_rn(amax, t6));
+// E4M3_RNE_satfinite(amax / (6 t)) decided on the exact quotient.  The estimate
+// amax * fl(1/fl(6t)) is within ~2 ulp, so the answer is s0 or a neighbour.
+__device__ __forceinline__ uint32_t block_scale_code(float amax, float t, float inv6t) {
+  uint32_t s = e4m3_rn_satfinite(__fmul_rn(amax, inv6t));
   if (s < 126u && scale_passes(amax, 0.5f * (e4m3_value(s) + e4m3_value(s + 1)), t, s + 1))
     s += 1;
   else if (s > 0u && !scale_passes(amax, 0.5f * (e4m3_value(s - 1) + e4m3_value(s)), t, s))
@@ -111,45 +118,61 @@ __device__ __forceinline__ uint32_t block_scale_code(float amax, float t, float 
   return s;
 }
 
-// Exact E2M1 magnitude of |x| (fp32 value of a bf16) for block scale S, tensor scale t.
-__device__ __noinline__ uint32_t e2m1_exact_pair(float ax_hi, float ax_lo, float S, float t) {
-  uint32_t mh = 0, ml = 0;
-  if (S > 0.f) {
-#pragma unroll
-    for (int i = 0; i < 7; ++i) {
-      const float P = __fmul_rn(c_e2m1_mid[i], S);         // exact: <= 7 significant bits
-      const float h = __fmul_rn(P, t);
-      const float e = __fmaf_rn(P, t, -h);                 // exact residual: threshold = h + e
-      const bool up_on_tie = (i & 1);
-      mh += (ax_hi > h || (ax_hi == h && (e < 0.f || (e == 0.f && up_on_tie)))) ? 1u : 0u;
-      ml += (ax_lo > h || (ax_lo == h && (e < 0.f || (e == 0.f && up_on_tie)))) ? 1u : 0u;
-    }
-  }
-  return (mh << 4) | ml;
+// Smallest bf16 (as bits) whose value passes E2M1 midpoint i of a block with
+// decode scale S t: value > mu_i S t, or equal with the tie going up (odd i).
+// h = fl(P t) with P = mu_i S exact, e = fma(P, t, -h) the exact residual.
+__device__ __forceinline__ uint32_t e2m1_threshold_bits(float P, float t, int i) {
+  const float h = __fmul_rn(P, t);
+  const float e = __fmaf_rn(P, t, -h);
+  const uint32_t hb = __float_as_uint(h);
+  if (isinf(h)) return 0x7F80u;
+  if (h == 0.f) return 1u;                                  // any positive value passes
+  if ((hb & 0xFFFFu) != 0u) return (hb >> 16) + 1u;         // next bf16 above h (and above h + e)
+  const uint32_t v0 = hb >> 16;                             // h is itself a bf16 value
+  if (e > 0.f) return v0 + 1u;
+  if (e < 0.f) return v0;
+  return (i & 1) ? v0 : v0 + 1u;                            // exact tie
 }
 
-// Codes for 4 bf16x2 words (8 elements) -> 32 bits of packed codes.
-template <bool kExact>
-__device__ __forceinline__ uint32_t codes8(const uint32_t (&w)[4], float inv_d, float S, float t) {
+__device__ __forceinline__ uint32_t e2m1_fast_code(uint32_t bf16_bits, float inv_d) {
+  const float v = __uint_as_float(bf16_bits << 16);
+  return e2m1x2_rn_satfinite(0.f, __fmul_rn(v, inv_d)) & 0xFu;
+}
+
+// Packed codes for 4 bf16x2 words (8 elements) -> 32 bits, fast path.
+__device__ __forceinline__ uint32_t codes8_fast(const uint32_t* w, float inv_d) {
   uint32_t out = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float alo = __uint_as_float((w[i] & 0x7FFFu) << 16);
     const float ahi = __uint_as_float(w[i] & 0x7FFF0000u);
-    uint32_t byte;
-    if (kExact) byte = e2m1_exact_pair(ahi, alo, S, t);
-    else byte = e2m1x2_rn_satfinite(__fmul_rn(ahi, inv_d), __fmul_rn(alo, inv_d));
+    uint32_t byte = e2m1x2_rn_satfinite(__fmul_rn(ahi, inv_d), __fmul_rn(alo, inv_d));
     byte |= ((w[i] >> 12) & 0x8u) | ((w[i] >> 24) & 0x80u);       // signs of x
     out |= byte << (8 * i);
   }
   return out;
 }
 
-__device__ __forceinline__ float resolve_tensor_scale(const float* t_in, const float* partial, int npartial) {
-  if (t_in != nullptr) return __ldg(t_in);
-  float m = 0.f;
-  for (int i = 0; i < npartial; ++i) m = fmaxf(m, __ldg(partial + i));
-  return m == 0.f ? 1.0f : __fdiv_rn(m, 2688.0f);
+// Exact path: count the thresholds each |x| reaches, two elements at a time
+// with packed bf16x2 compares (1.0 / 0.0) accumulated on top of 128.0, which
+// keeps the count in the low mantissa bits.
+__device__ __forceinline__ uint32_t codes8_exact(const uint32_t* w, const uint32_t (&B)[7]) {
+  uint32_t out = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t a = w[i] & 0x7FFF7FFFu;
+    uint32_t acc = 0x43004300u;
+#pragma unroll
+    for (int k = 0; k < 7; ++k) {
+      uint32_t ge;
+      asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(ge) : "r"(a), "r"(B[k]));
+      asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(acc) : "r"(acc), "r"(ge));
+    }
+    uint32_t byte = (acc & 0x7u) | ((acc >> 12) & 0x70u);
+    byte |= ((w[i] >> 12) & 0x8u) | ((w[i] >> 24) & 0x80u);
+    out |= byte << (8 * i);
+  }
+  return out;
 }
 
 // rows x K bf16 -> codes [rows, K/2], tiled scales, t.
@@ -158,10 +181,10 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(
     const float* __restrict__ partial, int npartial, uint2* __restrict__ codes,
     uint8_t* __restrict__ scales, float* __restrict__ t_out) {
   __shared__ float s_inv_d[128];
-  __shared__ uint8_t s_danger[128];
+  __shared__ uint32_t s_fast_ok[128];
+  __shared__ uint4 s_thr[128];                               // 7 thresholds (bf16 bits) + pad
   __shared__ float s_t;
   if (threadIdx.x < 32) {
-    // Every warp-0 lane reduces a slice of the partial maxima.
     float m = 0.f;
     if (t_in == nullptr)
       for (int i = threadIdx.x; i < npartial; i += 32) m = fmaxf(m, __ldg(partial + i));
@@ -175,60 +198,68 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(
   }
   __syncthreads();
   const float t = s_t;
+  // Per E4M3 scale code: the exact thresholds, and whether the fast path
+  // (fp32 quotient + cvt) provably agrees with them for every bf16 input: both
+  // are monotone in |x|, so agreeing on both sides of every exact threshold
+  // means agreeing everywhere.
   if (threadIdx.x < 127) {
-    const float S = e4m3_value(threadIdx.x);
-    const float d = __fmul_rn(S, t);
-    float inv = 0.f;
-    uint32_t danger = 0;
-    if (threadIdx.x != 0) {
-      inv = __frcp_rn(d);
-      if (!(d >= 1.17549435e-38f) || isinf(inv)) {
-        danger = 0x7F;                                      // tiny / huge: exact path
-      } else {
+    const uint32_t c = threadIdx.x;
+    const float S = e4m3_value(c);
+    uint32_t b[7];
 #pragma unroll
-        for (int i = 0; i < 7; ++i) {
-          const float h = __fmul_rn(__fmul_rn(c_e2m1_mid[i], S), t);
-          const uint32_t f = __float_as_uint(h) & 0xFFFFu;
-          const uint32_t dist = min(f, 0x10000u - f);        // fp32 ulps to the nearest bf16
-          if (dist <= 16u || !(h >= 1e-30f) || isinf(h)) danger |= 1u << i;
+    for (int i = 0; i < 7; ++i) b[i] = (c == 0) ? 0x7F80u : e2m1_threshold_bits(__fmul_rn(c_e2m1_mid[i], S), t, i);
+    const float d = __fmul_rn(S, t);
+    const float inv = (c == 0) ? 0.f : __frcp_rn(d);
+    bool ok = (c == 0) || (d >= 1.17549435e-38f && !isinf(inv));
+    if (c != 0 && ok) {
+#pragma unroll
+      for (int i = 0; i < 7; ++i) {
+        if (b[i] >= 0x7F80u) {
+          ok = ok && e2m1_fast_code(0x7F7Fu, inv) == (uint32_t)i;
+        } else {
+          ok = ok && e2m1_fast_code(b[i], inv) == (uint32_t)(i + 1);
+          if (b[i] > 0u) ok = ok && e2m1_fast_code(b[i] - 1u, inv) == (uint32_t)i;
         }
       }
     }
-    s_inv_d[threadIdx.x] = inv;
-    s_danger[threadIdx.x] = (uint8_t)danger;
+    s_inv_d[c] = inv;
+    s_fast_ok[c] = ok ? 1u : 0u;
+    s_thr[c] = make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16), b[6] | (0x7F80u << 16));
   }
   __syncthreads();
 
-  const float t6 = __fmul_rn(6.0f, t);
+  const float inv6t = __frcp_rn(__fmul_rn(6.0f, t));
   const uint32_t nbk = K >> 4;                               // 16-element blocks per row
   const uint32_t atoms_per_rowtile = K >> 6;
-  const uint64_t nblocks = (uint64_t)rows * nbk;
+  const uint32_t nblocks = rows * nbk;                       // < 2^32 (checked on the host)
   const uint32_t lane = threadIdx.x & 31u;
-  const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
-  for (uint64_t base = (uint64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31u); base < nblocks;
-       base += stride) {
-    const uint64_t b = base + lane;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t base = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); base < nblocks; base += stride) {
+    const uint32_t b = base + lane;
     const bool valid = b < nblocks;                          // nblocks % 4 == 0: groups of 4 agree
     uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (valid) {
-      const uint4 v0 = __ldg(x + 2 * b), v1 = __ldg(x + 2 * b + 1);
+      const uint4 v0 = __ldg(x + 2 * (size_t)b), v1 = __ldg(x + 2 * (size_t)b + 1);
       w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
       w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
     }
-    uint32_t m2 = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(w[0], w[1]), bf16x2_absmax(w[2], w[3])),
-                                bf16x2_absmax(bf16x2_absmax(w[4], w[5]), bf16x2_absmax(w[6], w[7])));
+    const uint32_t m2 = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(w[0], w[1]), bf16x2_absmax(w[2], w[3])),
+                                      bf16x2_absmax(bf16x2_absmax(w[4], w[5]), bf16x2_absmax(w[6], w[7])));
     const float amax = bf16x2_hmax_to_f32(m2);
-    const uint32_t s = block_scale_code(amax, t, t6);
-    const float inv_d = s_inv_d[s];
+    const uint32_t s = block_scale_code(amax, t, inv6t);
     uint2 c;
-    const uint32_t wa[4] = {w[0], w[1], w[2], w[3]}, wb[4] = {w[4], w[5], w[6], w[7]};
-    if (s_danger[s] == 0) {
-      c.x = codes8<false>(wa, inv_d, 0.f, t);
-      c.y = codes8<false>(wb, inv_d, 0.f, t);
+    if (s_fast_ok[s]) {
+      const float inv_d = s_inv_d[s];
+      c.x = codes8_fast(w, inv_d);
+      c.y = codes8_fast(w + 4, inv_d);
     } else {
-      const float S = e4m3_value(s);
-      c.x = codes8<true>(wa, inv_d, S, t);
-      c.y = codes8<true>(wb, inv_d, S, t);
+      const uint4 T = s_thr[s];
+      const uint32_t B[7] = {__byte_perm(T.x, 0, 0x1010), __byte_perm(T.x, 0, 0x3232),
+                             __byte_perm(T.y, 0, 0x1010), __byte_perm(T.y, 0, 0x3232),
+                             __byte_perm(T.z, 0, 0x1010), __byte_perm(T.z, 0, 0x3232),
+                             __byte_perm(T.w, 0, 0x1010)};
+      c.x = codes8_exact(w, B);
+      c.y = codes8_exact(w + 4, B);
     }
     // Gather the 4 scale bytes of an aligned group of 4 blocks (same row, same atom).
     uint32_t sv = s << (8 * (lane & 3u));
@@ -237,21 +268,20 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(
     if (valid) {
       codes[b] = c;
       if ((lane & 3u) == 0u) {
-        const uint32_t r = (uint32_t)(b / nbk), kb = (uint32_t)(b - (uint64_t)r * nbk);
-        const uint64_t off = ((uint64_t)(r >> 7) * atoms_per_rowtile + (kb >> 2)) * 512u +
-                             (r & 31u) * 16u + ((r & 127u) >> 5) * 4u;
+        const uint32_t r = b / nbk, kb = b - r * nbk;
+        const size_t off = ((size_t)(r >> 7) * atoms_per_rowtile + (kb >> 2)) * 512u + (r & 31u) * 16u +
+                           ((r & 127u) >> 5) * 4u;
         *reinterpret_cast<uint32_t*>(scales + off) = sv;
       }
     }
   }
   // Zero the scales of the padding rows up to the next multiple of 128.
   const uint32_t rows_pad = (rows + 127u) & ~127u;
-  const uint64_t npad = (uint64_t)(rows_pad - rows) * atoms_per_rowtile;
-  for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < npad; i += stride) {
-    const uint32_t r = rows + (uint32_t)(i / atoms_per_rowtile);
-    const uint32_t kt = (uint32_t)(i % atoms_per_rowtile);
-    const uint64_t off = ((uint64_t)(r >> 7) * atoms_per_rowtile + kt) * 512u + (r & 31u) * 16u +
-                         ((r & 127u) >> 5) * 4u;
+  const uint32_t npad = (rows_pad - rows) * atoms_per_rowtile;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < npad; i += stride) {
+    const uint32_t r = rows + i / atoms_per_rowtile;
+    const uint32_t kt = i % atoms_per_rowtile;
+    const size_t off = ((size_t)(r >> 7) * atoms_per_rowtile + kt) * 512u + (r & 31u) * 16u + ((r & 127u) >> 5) * 4u;
     *reinterpret_cast<uint32_t*>(scales + off) = 0u;
   }
 }

@@ -6,6 +6,7 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "../../include/nvq.h"
@@ -61,9 +62,10 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D row-major tensor map: inner dimension `inner` elements, `outer` rows,
-// row pitch `pitch_bytes`, box {box_inner, box_outer}, 128-byte swizzle.
+// row pitch `pitch_bytes`, box {box_inner, box_outer}.
 bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-                 uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+                 uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
@@ -71,45 +73,57 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uin
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 constexpr int64_t kMaxDim = (int64_t)1 << 31;
 
-// Decode split of K: enough warps to cover the SMs, only at small batch.
-uint32_t w4a16_splits(int64_t M, int64_t N, int64_t K) {
+// Decode work split: KS warps of a CTA share a 16-row tile (in-CTA K split, no
+// workspace); a global K split (FP32 partials + reduce kernel) only when the
+// weight matrix is too small to give ~1024 warps otherwise.
+struct W4a16Plan {
+  int nt8;          // batch tiles of 8 rows per pass
+  int ks;           // warps per row tile
+  uint32_t splits;  // global K splits
+};
+
+W4a16Plan w4a16_plan(int64_t M, int64_t N, int64_t K) {
+  W4a16Plan pl;
+  pl.nt8 = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
   const uint32_t G = (uint32_t)(K / 128);
-  if (M > 64) return 1;
   const uint64_t tiles = (uint64_t)(N / 16);
-  uint32_t best = 1;
-  for (uint32_t s = 1; s <= G; ++s) {
-    if (G % s) continue;
-    best = s;
-    if (tiles * s >= 2048) break;
+  const uint64_t want = 1024;
+  pl.ks = 1;
+  while (pl.ks < 4 && tiles * pl.ks < want && G % (2 * pl.ks) == 0) pl.ks *= 2;
+  pl.splits = 1;
+  if (M <= 64) {
+    while (tiles * pl.ks * pl.splits < want && G % (pl.ks * pl.splits * 2) == 0 && pl.splits < 16) pl.splits *= 2;
   }
-  return best;
+  return pl;
 }
 
-template <int NT8>
-nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* y, float* ws, int64_t M,
-                               int64_t N, int64_t K, uint32_t splits, cudaStream_t stream) {
+template <int NT8, int KS>
+nvq_status launch_w4a16_t(const void* x, const uint8_t* pc, const void* ps, void* y, float* ws, int64_t M,
+                          int64_t N, int64_t K, uint32_t splits, cudaStream_t stream) {
   using namespace nvq::w4a16;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(w4a16_kernel<NT8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)smem_bytes<NT8>());
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "w4a16_gemm: smem attribute");
   const uint32_t G = (uint32_t)(K / 128);
   const uint32_t gps = G / splits;
-  const uint32_t cta_rows = (uint32_t)((N / 16 + WARPS - 1) / WARPS);
-  const uint64_t grid = (uint64_t)cta_rows * splits;
-  w4a16_kernel<NT8><<<(unsigned)grid, THREADS, smem_bytes<NT8>(), stream>>>(
+  constexpr int RT = WARPS / KS;
+  const uint64_t cta_rows = (uint64_t)((N / 16 + RT - 1) / RT);
+  const uint64_t grid = cta_rows * splits;
+  w4a16_kernel<NT8, KS><<<(unsigned)grid, THREADS, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(x), reinterpret_cast<const uint4*>(pc), static_cast<const uint32_t*>(ps),
       static_cast<__nv_bfloat16*>(y), ws, (uint32_t)M, (uint32_t)N, (uint32_t)K, gps, splits);
   return launch_status("w4a16_kernel");
+}
+
+template <int NT8>
+nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* y, float* ws, int64_t M, int64_t N,
+                        int64_t K, const W4a16Plan& pl, cudaStream_t stream) {
+  if (pl.ks == 4) return launch_w4a16_t<NT8, 4>(x, pc, ps, y, ws, M, N, K, pl.splits, stream);
+  if (pl.ks == 2) return launch_w4a16_t<NT8, 2>(x, pc, ps, y, ws, M, N, K, pl.splits, stream);
+  return launch_w4a16_t<NT8, 1>(x, pc, ps, y, ws, M, N, K, pl.splits, stream);
 }
 
 }  // namespace
@@ -165,7 +179,7 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const flo
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (rows < 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_quantize: rows < 0 or K <= 0");
   if (K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize: K % 64 != 0");
-  if (rows >= kMaxDim || K >= kMaxDim || (rows * (K / 16)) >= ((int64_t)1 << 40))
+  if (rows >= kMaxDim || K >= kMaxDim || (rows * (K / 16)) >= ((int64_t)1 << 32))
     return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize: tensor too large");
   if (tensor_scale_out == nullptr) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_quantize: tensor_scale_out is NULL");
   if (rows > 0 && (x_bf16 == nullptr || codes == nullptr || scales == nullptr))
@@ -199,27 +213,23 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const flo
 }
 
 // ------------------------------------------------------------------ NVFP4 GEMM
-nvq_status nvfp4_gemm_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const float* t_x,
-                           const uint8_t* w_codes, const uint8_t* w_scales, const float* t_w, void* y_bf16,
-                           int64_t M, int64_t N, int64_t K, void* stream_) {
+}  // extern "C"
+
+namespace {
+
+template <int BN>
+nvq_status launch_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const float* t_x, const uint8_t* w_codes,
+                       const uint8_t* w_scales, const float* t_w, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                       cudaStream_t stream) {
   using namespace nvq::w4a4;
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4: bad sizes");
-  if (N % 8 != 0 || K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4: need N % 8 == 0, K % 64 == 0");
-  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4: too large");
-  if (!x_codes || !x_scales || !t_x || !w_codes || !w_scales || !t_w || !y_bf16)
-    return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4: NULL pointer");
-  if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
-      !aligned16(y_bf16) || (reinterpret_cast<uintptr_t>(t_x) & 3u) || (reinterpret_cast<uintptr_t>(t_w) & 3u))
-    return fail(NVQ_ERR_MISALIGNED, "nvfp4_gemm_w4a4: pointer not aligned");
-  if (M == 0) return NVQ_OK;
+  using C = Cfg<BN>;
   CUtensorMap ma, mb, my;
   if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
                    BKB, BM) ||
       !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
                    BKB, BN) ||
       !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2,
-                   C_CHUNK_COLS, BM))
+                   C_COLS, BM, CU_TENSOR_MAP_SWIZZLE_64B))
     return fail(NVQ_ERR_CUDA, "nvfp4_gemm_w4a4: tensor map encoding failed");
   Params p;
   p.x_scales = x_scales;
@@ -237,13 +247,37 @@ nvq_status nvfp4_gemm_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, cons
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    attr_err = cudaFuncSetAttribute(nvfp4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "nvfp4_gemm_w4a4: smem attribute");
   const uint64_t tiles = (uint64_t)p.num_m_tiles * p.num_n_tiles;
   const int grid = (int)std::min<uint64_t>(tiles, (uint64_t)sm_count());
-  nvfp4_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, my, p);
+  nvfp4_gemm_kernel<BN><<<grid, THREADS, C::SMEM_BYTES, stream>>>(ma, mb, my, p);
   return launch_status("nvfp4_gemm_kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+nvq_status nvfp4_gemm_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const float* t_x,
+                           const uint8_t* w_codes, const uint8_t* w_scales, const float* t_w, void* y_bf16,
+                           int64_t M, int64_t N, int64_t K, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4: bad sizes");
+  if (N % 8 != 0 || K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4: need N % 8 == 0, K % 64 == 0");
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4: too large");
+  if (!x_codes || !x_scales || !t_x || !w_codes || !w_scales || !t_w || !y_bf16)
+    return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4: NULL pointer");
+  if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(y_bf16) || (reinterpret_cast<uintptr_t>(t_x) & 3u) || (reinterpret_cast<uintptr_t>(t_w) & 3u))
+    return fail(NVQ_ERR_MISALIGNED, "nvfp4_gemm_w4a4: pointer not aligned");
+  if (M == 0) return NVQ_OK;
+  // 192-wide N tiles: two accumulators (384 TMEM columns) fit beside the scales,
+  // and every tile starts at a row offset that is a multiple of 64 within its
+  // 128-row scale atom, so the B-scale TMEM address moves by 0 or 2 columns.
+  return launch_w4a4<192>(x_codes, x_scales, t_x, w_codes, w_scales, t_w, y_bf16, M, N, K, stream);
 }
 
 // ------------------------------------------------------------------ INT4
@@ -289,8 +323,8 @@ nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int6
 // ------------------------------------------------------------------ W4A16 decode GEMM
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0 || N % 16 || K % 128) return 0;
-  const uint32_t s = w4a16_splits(M, N, K);
-  return s <= 1 ? 0 : (size_t)s * (size_t)M * (size_t)N * sizeof(float);
+  const W4a16Plan pl = w4a16_plan(M, N, K);
+  return pl.splits <= 1 ? 0 : (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(float);
 }
 
 nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const void* packed_scales, void* y_bf16,
@@ -303,23 +337,23 @@ nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const voi
   if (!x_bf16 || !packed_codes || !packed_scales || !y_bf16) return fail(NVQ_ERR_INVALID_ARG, "w4a16_gemm: NULL pointer");
   if (!aligned16(x_bf16) || !aligned16(packed_codes) || !aligned16(packed_scales) || !aligned16(y_bf16))
     return fail(NVQ_ERR_MISALIGNED, "w4a16_gemm: pointer not 16-byte aligned");
-  const uint32_t splits = w4a16_splits(M, N, K);
+  const W4a16Plan pl = w4a16_plan(M, N, K);
   float* ws = nullptr;
-  if (splits > 1) {
-    const size_t need = (size_t)splits * (size_t)M * (size_t)N * sizeof(float);
+  if (pl.splits > 1) {
+    const size_t need = (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(float);
     if (workspace == nullptr || workspace_bytes < need) return fail(NVQ_ERR_WORKSPACE, "w4a16_gemm: workspace too small");
     if (!aligned16(workspace)) return fail(NVQ_ERR_MISALIGNED, "w4a16_gemm: workspace not 16-byte aligned");
     ws = static_cast<float*>(workspace);
   }
   nvq_status st;
-  if (M <= 8) st = launch_w4a16<1>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, splits, stream);
-  else if (M <= 16) st = launch_w4a16<2>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, splits, stream);
-  else st = launch_w4a16<4>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, splits, stream);
-  if (st != NVQ_OK || splits == 1) return st;
+  if (pl.nt8 == 1) st = launch_w4a16<1>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, pl, stream);
+  else if (pl.nt8 == 2) st = launch_w4a16<2>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, pl, stream);
+  else st = launch_w4a16<4>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, pl, stream);
+  if (st != NVQ_OK || pl.splits == 1) return st;
   const uint64_t n4 = (uint64_t)M * (uint64_t)N / 4;
   const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>((n4 + 255) / 256, (uint64_t)sm_count() * 8));
   nvq::w4a16::w4a16_reduce_kernel<<<grid, 256, 0, stream>>>(static_cast<const float4*>(workspace),
-                                                            static_cast<uint2*>(y_bf16), splits, n4);
+                                                            static_cast<uint2*>(y_bf16), pl.splits, n4);
   return launch_status("w4a16_reduce_kernel");
 }
 

@@ -1,0 +1,72 @@
+"""Run one library call on one shape a few times, for profilers (ncu) and quick timing.
+
+  python -m phase_disaggregated_quantized_b200.profile_case --op gemm --M 8192 --K 4096 --N 24576
+  python -m phase_disaggregated_quantized_b200.profile_case --op w4a16 --M 1 --K 4096 --N 24576
+  python -m phase_disaggregated_quantized_b200.profile_case --op quantize --M 8192 --K 12288
+
+Inputs are drawn on the GPU from the seeded generators; the offline steps
+(weight quantization and reorder) run once before the measured calls.  Prints
+the mean CUDA-event time per call of the measured op.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+import phase_disaggregated_quantized_b200 as nvq
+from phase_disaggregated_quantized_b200 import synth
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--op", choices=("gemm", "w4a16", "quantize"), required=True)
+    ap.add_argument("--M", type=int, required=True)
+    ap.add_argument("--K", type=int, required=True)
+    ap.add_argument("--N", type=int, default=0)
+    ap.add_argument("--iters", type=int, default=3)
+    a = ap.parse_args()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    x = synth.activations_cuda(a.M, a.K, seed=11, device=dev)
+    if a.op == "gemm":
+        w = synth.weights_cuda(a.N, a.K, seed=11, device=dev)
+        wq = nvq.nvfp4_quantize(w)
+        xq = nvq.nvfp4_quantize(x)
+        y = torch.empty(a.M, a.N, dtype=torch.bfloat16, device=dev)
+        run = lambda: nvq.nvfp4_gemm_w4a4(xq, wq, a.M, a.N, a.K, y=y)  # noqa: E731
+        work = 2.0 * a.M * a.N * a.K
+        unit = "TFLOP/s"
+    elif a.op == "w4a16":
+        w = synth.weights_cuda(a.N, a.K, seed=11, device=dev)
+        codes, scales = nvq.int4_quantize(w)
+        pc, ps = nvq.int4_pack_weights(codes, scales, a.N, a.K)
+        y = torch.empty(a.M, a.N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(16, nvq.w4a16_workspace_bytes(a.M, a.N, a.K)), dtype=torch.uint8, device=dev)
+        run = lambda: nvq.w4a16_gemm(x, pc, ps, a.N, y=y, workspace=ws)  # noqa: E731
+        work = a.N * a.K / 2 + 2 * a.N * a.K / 128 + 2 * a.M * a.K + 2 * a.M * a.N
+        unit = "GB/s"
+    else:
+        codes = torch.empty(a.M, a.K // 2, dtype=torch.uint8, device=dev)
+        sc = torch.empty(nvq.nvfp4_scales_bytes(a.M, a.K), dtype=torch.uint8, device=dev)
+        t = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.empty(nvq.nvfp4_quantize_workspace_bytes(a.M, a.K), dtype=torch.uint8, device=dev)
+        run = lambda: nvq.nvfp4_quantize(x, None, codes=codes, scales=sc, tensor_scale_out=t, workspace=ws)  # noqa
+        work = 2.0 * a.M * a.K * 2 + a.M * a.K * (0.5 + 1 / 16)
+        unit = "GB/s"
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.iters):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    nvq.check_device_error()
+    s = e0.elapsed_time(e1) / 1e3 / a.iters
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    print(f"{a.op} M={a.M} K={a.K} N={a.N}: {1e6 * s:.2f} us/call, {work / s / scale:.1f} {unit}")
+
+
+if __name__ == "__main__":
+    main()

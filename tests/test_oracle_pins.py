@@ -318,11 +318,12 @@ def test_int4_reorder_is_bijection_and_hand_slots():
     u2, s2 = int4.unpack_weights(pc, ps, N, K)
     assert np.array_equal(u, u2) and np.array_equal(s, s2)
     words = pc.view("<u4")
-    # unit 0, word 0 (lane 0, j 0): nibbles (0,0) (8,0) (0,8) (8,8) (0,1) (8,1) (0,9) (8,9)
-    want = [u[0, 0], u[8, 0], u[0, 8], u[8, 8], u[0, 1], u[8, 1], u[0, 9], u[8, 9]]
+    # unit 0, word 0 (lane 0, j 0): nibbles (0,0) (8,0) (0,2) (8,2) (0,1) (8,1) (0,3) (8,3)
+    want = [u[0, 0], u[8, 0], u[0, 2], u[8, 2], u[0, 1], u[8, 1], u[0, 3], u[8, 3]]
     assert [(int(words[0]) >> (4 * p)) & 15 for p in range(8)] == [int(v) for v in want]
-    # lane 5 (g=1, c=1), j = 6 -> word 128 + 4*5 + 2, nibble 0 = (1, 16*6 + 2)
-    assert (int(words[128 + 22]) & 15) == u[1, 98]
+    # lane 5 (g=1, c=1), j = 6 -> word 128 + 4*5 + 2, nibble 0 = (1, 32*1 + 4*6), nibble 7 = (9, 59)
+    assert (int(words[128 + 22]) & 15) == u[1, 56]
+    assert (int(words[128 + 22]) >> 28) == u[9, 59]
     # unit 1 = tile 0, group 1: its word 0 nibble 0 is (0, 128)
     assert (int(words[256]) & 15) == u[0, 128]
     sw = ps.view("<u2")
