@@ -100,6 +100,29 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K,
                           void* stream);
 
 /* ------------------------------------------------------------------------ *
+ * nvfp4_quantize without any device allocation or workspace (no counterpart
+ * on the pages; an addition of this library).  For callers that cannot call
+ * cudaMalloc or lend scratch memory: for example an engine whose device memory
+ * is all owned by its own pool once serving starts, or a plugin that must not
+ * allocate behind its host's back.  Same arguments, same results (bit for bit)
+ * as nvfp4_quantize, minus the workspace.
+ *
+ * The tensor-amax partials live in a fixed 4 KiB file-scope device array
+ * inside the library (1024 floats, one partial per 2^20 input elements), held
+ * on every GPU that loads the library until the process exits.  Limit:
+ * rows * K <= 2^30 elements; larger calls return NVQ_ERR_UNSUPPORTED_SHAPE.
+ * The first call on each device resolves the array's device address with
+ * cudaGetSymbolAddress (that device must be current); make that first call
+ * before any stream capture.  All calls on a device share the array: calls
+ * that overlap on the GPU (different streams, no ordering) race and give wrong
+ * results.  Each call overwrites every partial it later reads, so nothing
+ * needs clearing between calls.  Calls no cudaMalloc/cudaFree.
+ * ------------------------------------------------------------------------ */
+nvq_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t K,
+                                  const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,
+                                  float* tensor_scale_out, void* stream);
+
+/* ------------------------------------------------------------------------ *
  * NVFP4 W4A4 GEMM (Mix-Quant page, section 2.3: the prefill worker's W4A4 path).
  *
  *   Y[m, n] = bf16_RNE( t_x * t_w * sum_k (e4m3(sx[m, k/16]) e2m1(cx[m, k]))

@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
             "nvfp4_scales_bytes": ([i64, i64], sz),
             "nvfp4_quantize_workspace_bytes": ([i64, i64], sz),
             "nvfp4_quantize": ([vp, i64, i64, vp, vp, vp, vp, vp, sz, vp], i32),
+            "nvfp4_quantize_noalloc": ([vp, i64, i64, vp, vp, vp, vp, vp], i32),
             "nvfp4_gemm_w4a4": ([vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
             "int4_quantize": ([vp, i64, i64, vp, vp, vp], i32),
             "int4_pack_weights": ([vp, vp, i64, i64, vp, vp, vp], i32),
@@ -129,6 +130,17 @@ def nvfp4_quantize(x, tensor_scale_in=None, *, codes=None, scales=None, tensor_s
     _check(lib().nvfp4_quantize(_ptr(x), rows, K, _ptr(tensor_scale_in), _ptr(codes), _ptr(scales),
                                 _ptr(tensor_scale_out), _ptr(workspace), ws_bytes, _stream(stream)),
            "nvfp4_quantize")
+    return codes, scales, tensor_scale_out
+
+
+def nvfp4_quantize_noalloc(x, tensor_scale_in=None, *, codes, scales, tensor_scale_out, stream=None):
+    """nvfp4_quantize for callers that cannot allocate: the library uses its own
+    fixed device scratch (rows * K <= 2^30), so all outputs must be passed in."""
+    _need_cuda(x, tensor_scale_in, codes, scales, tensor_scale_out)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+    rows, K = x.shape
+    _check(lib().nvfp4_quantize_noalloc(_ptr(x), rows, K, _ptr(tensor_scale_in), _ptr(codes), _ptr(scales),
+                                        _ptr(tensor_scale_out), _stream(stream)), "nvfp4_quantize_noalloc")
     return codes, scales, tensor_scale_out
 
 

@@ -173,6 +173,64 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K) {
   return (size_t)nvq::kAmaxMaxBlocks * sizeof(float);
 }
 
+}  // extern "C"
+
+namespace {
+
+nvq_status quantize_validate(const char* name, const void* x_bf16, int64_t rows, int64_t K, uint8_t* codes,
+                             uint8_t* scales, float* tensor_scale_out) {
+  char msg[160];
+  if (rows < 0 || K <= 0) {
+    snprintf(msg, sizeof(msg), "%s: rows < 0 or K <= 0", name);
+    return fail(NVQ_ERR_INVALID_ARG, msg);
+  }
+  if (K % 64 != 0) {
+    snprintf(msg, sizeof(msg), "%s: K %% 64 != 0", name);
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, msg);
+  }
+  if (rows >= kMaxDim || K >= kMaxDim || (rows * (K / 16)) >= ((int64_t)1 << 32)) {
+    snprintf(msg, sizeof(msg), "%s: tensor too large", name);
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, msg);
+  }
+  if (tensor_scale_out == nullptr) {
+    snprintf(msg, sizeof(msg), "%s: tensor_scale_out is NULL", name);
+    return fail(NVQ_ERR_INVALID_ARG, msg);
+  }
+  if (rows > 0 && (x_bf16 == nullptr || codes == nullptr || scales == nullptr)) {
+    snprintf(msg, sizeof(msg), "%s: NULL tensor pointer", name);
+    return fail(NVQ_ERR_INVALID_ARG, msg);
+  }
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales)) {
+    snprintf(msg, sizeof(msg), "%s: pointer not 16-byte aligned", name);
+    return fail(NVQ_ERR_MISALIGNED, msg);
+  }
+  return NVQ_OK;
+}
+
+// amax pre-pass (when t is not given) into `partial[0 .. amax_blocks)`, then the quantize pass.
+nvq_status quantize_launch(const void* x_bf16, int64_t rows, int64_t K, const float* tensor_scale_in, uint8_t* codes,
+                           uint8_t* scales, float* tensor_scale_out, float* partial, int amax_blocks,
+                           cudaStream_t stream) {
+  if (amax_blocks > 0) {
+    const size_t nvec = (size_t)rows * (size_t)K / 8;
+    nvq::nvfp4_amax_kernel<<<amax_blocks, nvq::kAmaxThreads, 0, stream>>>(static_cast<const uint4*>(x_bf16), nvec,
+                                                                           partial);
+    nvq_status st = launch_status("nvfp4_amax_kernel");
+    if (st != NVQ_OK) return st;
+  }
+  const uint64_t nblocks = (uint64_t)rows * (uint64_t)(K / 16);
+  const uint64_t want = (nblocks + nvq::kQuantThreads - 1) / nvq::kQuantThreads;
+  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count() * 8));
+  nvq::nvfp4_quantize_kernel<<<grid, nvq::kQuantThreads, 0, stream>>>(
+      static_cast<const uint4*>(x_bf16), (uint32_t)rows, (uint32_t)K, tensor_scale_in, partial, amax_blocks,
+      reinterpret_cast<uint2*>(codes), scales, tensor_scale_out);
+  return launch_status("nvfp4_quantize_kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
 nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const float* tensor_scale_in,
                           uint8_t* codes, uint8_t* scales, float* tensor_scale_out, void* workspace,
                           size_t workspace_bytes, void* stream_) {
@@ -355,6 +413,65 @@ nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const voi
   nvq::w4a16::w4a16_reduce_kernel<<<grid, 256, 0, stream>>>(static_cast<const float4*>(workspace),
                                                             static_cast<uint2*>(y_bf16), pl.splits, n4);
   return launch_status("w4a16_reduce_kernel");
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ NVFP4 quantize without allocation
+// For callers that cannot allocate device memory or lend a workspace: the amax
+// partials live in this fixed file-scope array instead.  Every GPU that loads
+// the library holds it (4 KiB) until the process exits.  All calls on a device
+// share it, so calls that overlap on the GPU race; each call overwrites every
+// slot it reads, so nothing has to be cleared between calls.
+namespace {
+
+constexpr int kNoallocPartials = 1024;                   // scratch capacity (floats)
+constexpr int64_t kNoallocElemsPerPartial = (int64_t)1 << 20;
+constexpr int kNoallocMaxDevices = 64;
+
+static __device__ __align__(256) float g_noalloc_amax_partials[kNoallocPartials];
+
+std::mutex g_noalloc_mutex;
+float* g_noalloc_scratch[kNoallocMaxDevices] = {};
+
+// Device address of the scratch array on the current device, resolved once per
+// device (with that device current) and cached.
+nvq_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "nvfp4_quantize_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= kNoallocMaxDevices) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: device ordinal >= 64");
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_scratch[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_amax_partials);
+    if (e != cudaSuccess) return cuda_fail(e, "nvfp4_quantize_noalloc: cudaGetSymbolAddress");
+    g_noalloc_scratch[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_noalloc_scratch[dev];
+  return NVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nvq_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t K, const float* tensor_scale_in,
+                                  uint8_t* codes, uint8_t* scales, float* tensor_scale_out, void* stream_) {
+  nvq_status st = quantize_validate("nvfp4_quantize_noalloc", x_bf16, rows, K, codes, scales, tensor_scale_out);
+  if (st != NVQ_OK) return st;
+  if (rows * K > (int64_t)kNoallocPartials * kNoallocElemsPerPartial)
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE,
+                "nvfp4_quantize_noalloc: rows*K exceeds 2^30 elements (the fixed scratch holds 1024 partial maxima, "
+                "one per 2^20 elements); use nvfp4_quantize with a workspace");
+  float* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != NVQ_OK) return st;
+  int amax_blocks = 0;
+  if (tensor_scale_in == nullptr && rows > 0)
+    amax_blocks = (int)((rows * K + kNoallocElemsPerPartial - 1) / kNoallocElemsPerPartial);
+  return quantize_launch(x_bf16, rows, K, tensor_scale_in, codes, scales, tensor_scale_out, scratch, amax_blocks,
+                         static_cast<cudaStream_t>(stream_));
 }
 
 }  // extern "C"
