@@ -4,69 +4,73 @@
 //
 //   Y[m, n] = bf16( t_x t_w sum_k sx[m, k/16] e2m1(cx[m, k]) * sw[n, k/16] e2m1(cw[n, k]) )
 //
-// Design (one CTA per SM, persistent over 128 x BN output tiles, BN = 192):
-//   warp 0      TMA producer: per k-stage of 256 elements it loads the A tile
-//               (128 rows x 128 bytes, 128B-swizzled), the B tile (BN x 128 B)
-//               and the 512-byte scale atoms covering those rows (plain bulk copies).
-//   warp 1      MMA issuer: for each 64-wide k step copies that step's scales
-//               into TMEM (tcgen05.cp 32x128b.warpx4, two alternating regions)
-//               and issues one tcgen05.mma.kind::mxf4nvf4.block_scale.block16
-//               (128 x BN x 64) into one of two FP32 TMEM accumulators; a
-//               tcgen05.commit frees each smem stage when its MMAs are done and
-//               marks an accumulator full after a tile's last k step.
-//   warps 2..5  epilogue: per accumulator, 32-column chunks are read with
-//               tcgen05.ld, scaled by t_x t_w, rounded to bf16, staged in 64B-
-//               swizzled smem and TMA-stored; the accumulator is released after
-//               the last chunk is read, so the next-but-one tile can reuse it
-//               while this tile's stores drain.  Two accumulators let the MMAs
-//               of tile i+1 run during the epilogue of tile i.
-// TMEM (512 columns): accumulators [0, BN) and [BN, 2 BN); the rest is a ring of
-// 12-column scale slots, one per MMA (A scales 4 columns, B scales 2 atoms x 4),
-// so a slot is rewritten only several MMAs after the MMA that read it.
-// The B-scale address is shifted by (n0 % 128) / 32 columns so that column j
-// holds tile rows 32 j .. 32 j + 31.  That shift must be even (a 224-wide tile,
-// whose shifts include 1 and 3, raised a misaligned-address error), so BN is a
-// multiple of 64.
+// Measured on B200: a block-scaled MMA instruction (M = 128, K = 64) takes about
+// the same issue time for N = 64 ... 256, a tcgen05.cp of scales placed in the
+// MMA thread's stream costs about a third of an MMA, and so does a per-MMA
+// handshake with another warp.  So the kernel uses the widest tile (128 x 256
+// per MMA) and keeps the MMA thread to waits, MMAs and commits:
+//
+//   warp 0       TMA producer: per 256-element k-stage, A (128 rows x 128 B) and
+//                B (256 rows x 128 B) with 128-byte swizzle, plus the 512-byte
+//                scale atoms (A: 4, B: 2 row-atoms x 4) as plain bulk copies.
+//   warp 1       MMA issuer: per k-stage one wait for the stage's data and one
+//                for its scales in TMEM, four tcgen05.mma.kind::mxf4nvf4
+//                .block_scale.block16 (128 x 256 x 64), two commits.
+//   warps 2..9   epilogue, two warps per TMEM sub-partition, each draining one
+//                64-column chunk after another (tcgen05.ld), scaling by t_x t_w,
+//                rounding to bf16 and TMA-storing its own 32 rows x 64 columns
+//                from its own 128-byte-swizzled staging buffer.
+//   warps 10..13 scale writers: per k-stage, read the stage's scales from shared
+//                memory and write them into a TMEM scale slot with tcgen05.st
+//                (each warp its own 32 lanes), then signal the MMA warp once.
+//
+// TMEM (512 columns): accumulator 0 = [0, 256), accumulator 1 = [128, 384); the
+// two overlap in [128, 256).  For each tile the epilogue reads the overlapping
+// 128 columns first and releases them before converting anything, so the next
+// tile's MMAs (other accumulator) wait only for that read; the rest of the
+// drain overlaps them.  [384, 480) holds two 48-column scale slots, one per
+// k-stage in flight: k step j uses A scales at columns 4j..4j+3 (column c: rows
+// 32c + lane) and B scales at 16 + 8j .. 16 + 8j + 7 (column c: rows 32c + lane),
+// the same in all four sub-partitions.
 #pragma once
 #include "ptx.cuh"
 
 namespace nvq {
 namespace w4a4 {
 
-constexpr int BM = 128;
+constexpr int BM = 128, BN = 256;
 constexpr int BKB = 128;                      // k-stage width in bytes (256 FP4 elements)
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int A_BYTES = BM * BKB;             // 16 KB
-constexpr int SFA_BYTES = 4 * 512;            // 4 k-atoms of 128 rows
-constexpr int SFB_ATOMS = 2;                  // 128-row scale atoms a 192-row B tile can touch
-constexpr uint32_t SF_SLOT_COLS = 12;         // A: 4 columns, B: 2 atoms x 4 columns
-constexpr int SFB_BYTES = SFB_ATOMS * 4 * 512;
-constexpr int C_COLS = 32;                    // epilogue chunk: 32 bf16 = 64-byte rows
-constexpr int C_BYTES = BM * C_COLS * 2;      // 8 KB per staging buffer
-constexpr int THREADS = 192;
+constexpr int B_BYTES = BN * BKB;             // 32 KB
+constexpr int SFA_BYTES = 4 * 512;            // 4 k-atoms of the 128 A rows
+constexpr int SFB_BYTES = 2 * 4 * 512;        // 2 row-atoms x 4 k-atoms of the 256 B rows
+constexpr int EPI_WARPS = 8;
+constexpr int C_COLS = 64;                    // epilogue chunk: 64 bf16 = 128-byte rows
+constexpr int C_BYTES = 32 * C_COLS * 2;      // 4 KB staging per epilogue warp (32 rows)
+constexpr int THREADS = (2 + EPI_WARPS + 4) * 32;   // 14 warps
 constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC1_COL = 128;            // accumulator 1 starts here (overlaps 0 by 128)
+constexpr uint32_t SF_COL0 = 384;
+constexpr uint32_t SF_SLOT_COLS = 48;         // one k-stage: 4 x (4 A + 8 B) columns
+constexpr uint32_t SF_SLOTS = 2;
 
-template <int BN>
-struct Cfg {
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 192, "BN: multiple of 64, two accumulators in TMEM");
-  static constexpr int B_BYTES = BN * BKB;
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_SFA = OFF_C + 2 * C_BYTES;
-  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-  static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 5;   // full, empty, acc_full x2, acc_empty x2, drain
-  static constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;    // + slack for 1024-byte alignment
-  static constexpr uint32_t SF_COL0 = 2 * BN;
-  static constexpr uint32_t SF_SLOTS = (TMEM_COLS - SF_COL0) / SF_SLOT_COLS;
-  // Instruction descriptor, kind::mxf4nvf4: A/B E2M1 (format 1), K-major,
-  // UE4M3 scales, N >> 3 in bits 17..22, M >> 4 in bits 24..28.
-  static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-  static_assert(SF_SLOTS >= 4, "TMEM budget");
-  static_assert(SMEM_BYTES <= 232448, "smem budget");
-};
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
+constexpr int OFF_SFA = OFF_C + EPI_WARPS * C_BYTES;
+constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+// full[S], empty[S], acc_full[2], acc_empty[2], overlap_free, sf_full[2], sf_free[2], drain
+constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 1 + 2 * SF_SLOTS + 1;
+constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
+constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;    // + slack for 1024-byte alignment
+static_assert(SMEM_BYTES <= 232448, "smem budget");
+static_assert(SF_COL0 + SF_SLOTS * SF_SLOT_COLS <= TMEM_COLS && ACC1_COL + BN <= SF_COL0, "TMEM budget");
+
+// Instruction descriptor, kind::mxf4nvf4: A/B E2M1 (format 1), K-major,
+// UE4M3 scales, N >> 3 in bits 17..22, M >> 4 in bits 24..28.
+constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
 struct Params {
   const uint8_t* x_scales;
@@ -79,21 +83,24 @@ struct Params {
   uint32_t n_row_atoms;    // padded N / 128
 };
 
-template <int BN>
+__device__ __forceinline__ uint32_t acc_col(uint32_t buf) { return buf ? ACC1_COL : 0u; }
+
 __global__ void __launch_bounds__(THREADS, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                   const __grid_constant__ CUtensorMap tmap_y, const Params p) {
-  using C = Cfg<BN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
-  const uint32_t bar_full = sbase + C::OFF_BAR;              // + 8 s
-  const uint32_t bar_empty = bar_full + 8 * STAGES;          // + 8 s
-  const uint32_t bar_acc_full = bar_empty + 8 * STAGES;      // + 8 b
-  const uint32_t bar_acc_empty = bar_acc_full + 16;          // + 8 b
-  const uint32_t bar_drain = bar_acc_empty + 16;
-  uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_PTR);
+  const uint32_t bar_full = sbase + OFF_BAR;                  // + 8 s
+  const uint32_t bar_empty = bar_full + 8 * STAGES;           // + 8 s
+  const uint32_t bar_acc_full = bar_empty + 8 * STAGES;       // + 8 b
+  const uint32_t bar_acc_empty = bar_acc_full + 16;           // + 8 b
+  const uint32_t bar_overlap = bar_acc_empty + 16;
+  const uint32_t bar_sf_full = bar_overlap + 8;               // + 8 slot
+  const uint32_t bar_sf_free = bar_sf_full + 8 * SF_SLOTS;    // + 8 slot
+  const uint32_t bar_drain = bar_sf_free + 8 * SF_SLOTS;
+  uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(smem + OFF_TMEM_PTR);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -102,7 +109,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_acc_full + 8 * b, 1);
-      mbar_init(bar_acc_empty + 8 * b, 4);                   // one arrive per epilogue warp
+      mbar_init(bar_acc_empty + 8 * b, EPI_WARPS);            // one arrive per epilogue warp
+    }
+    mbar_init(bar_overlap, EPI_WARPS);
+    for (uint32_t k = 0; k < SF_SLOTS; ++k) {
+      mbar_init(bar_sf_full + 8 * k, 4);                      // one arrive per scale-writer warp
+      mbar_init(bar_sf_free + 8 * k, 1);                      // one commit per k-stage from the MMA thread
     }
     mbar_init(bar_drain, 1);
     fence_mbar_init();
@@ -125,26 +137,24 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     if (lane == 0) {
       const uint64_t pol = policy_evict_last();
       uint32_t stage = 0, phase = 0;
-      uint32_t pending = 0, pending_parity = 0;              // per-stage bit masks
+      uint32_t pending = 0, pending_parity = 0;               // per-stage bit masks
       bool ok = true;
       for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const uint32_t mt = tile % p.num_m_tiles, nt = tile / p.num_m_tiles;
-        const uint32_t n0 = nt * BN;
-        const uint32_t atom0 = n0 / 128;
-        const uint32_t nb_atoms = min((uint32_t)SFB_ATOMS, min(p.n_row_atoms, (n0 + BN - 1) / 128 + 1) - atom0);
+        const uint32_t nb_atoms = min(2u, p.n_row_atoms - 2 * nt);
         for (uint32_t ks = 0; ks < p.num_k_stages; ++ks) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
           const uint32_t natoms = min(4u, p.k_atoms - 4 * ks);
-          const uint32_t bytes = A_BYTES + C::B_BYTES + natoms * 512u * (1u + nb_atoms);
+          const uint32_t bytes = A_BYTES + B_BYTES + natoms * 512u * (1u + nb_atoms);
           const uint32_t fb = bar_full + 8 * stage;
           mbar_arrive_expect_tx(fb, bytes);
-          tma_load_2d(sbase + C::OFF_A + stage * A_BYTES, &tmap_a, fb, (int)(ks * BKB), (int)(mt * BM), pol);
-          tma_load_2d(sbase + C::OFF_B + stage * C::B_BYTES, &tmap_b, fb, (int)(ks * BKB), (int)n0, pol);
-          bulk_load(sbase + C::OFF_SFA + stage * SFA_BYTES,
+          tma_load_2d(sbase + OFF_A + stage * A_BYTES, &tmap_a, fb, (int)(ks * BKB), (int)(mt * BM), pol);
+          tma_load_2d(sbase + OFF_B + stage * B_BYTES, &tmap_b, fb, (int)(ks * BKB), (int)(nt * BN), pol);
+          bulk_load(sbase + OFF_SFA + stage * SFA_BYTES,
                     p.x_scales + ((size_t)mt * p.k_atoms + 4 * ks) * 512u, natoms * 512u, fb);
           for (uint32_t a = 0; a < nb_atoms; ++a)
-            bulk_load(sbase + C::OFF_SFB + stage * SFB_BYTES + a * 2048u,
-                      p.w_scales + ((size_t)(atom0 + a) * p.k_atoms + 4 * ks) * 512u, natoms * 512u, fb);
+            bulk_load(sbase + OFF_SFB + stage * SFB_BYTES + a * 2048u,
+                      p.w_scales + ((size_t)(2 * nt + a) * p.k_atoms + 4 * ks) * 512u, natoms * 512u, fb);
           pending |= 1u << stage;
           pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -157,63 +167,37 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Kept lean: a single thread issues every tcgen05 instruction, so its
-    // instruction count per 64-wide K step bounds the tensor-pipe rate.  All
-    // descriptors are built once; per stage and step only the start-address
-    // field (low word, in 16-byte units) moves.
-    const uint64_t adesc0 = smem_desc(sbase + C::OFF_A, 0, 1024, kSwizzle128B);
-    const uint64_t bdesc0 = smem_desc(sbase + C::OFF_B, 0, 1024, kSwizzle128B);
-    const uint64_t sfadesc0 = smem_desc(sbase + C::OFF_SFA, 0, 128, kSwizzleNone);
-    const uint64_t sfbdesc0 = smem_desc(sbase + C::OFF_SFB, 0, 128, kSwizzleNone);
-    const uint32_t sf_begin = tmem_base + C::SF_COL0;
-    const uint32_t sf_end = sf_begin + C::SF_SLOTS * SF_SLOT_COLS;
-    uint32_t sf = sf_begin;                                  // next scale slot (ring)
-    uint32_t stage = 0, phase = 0, acc_par = 0;              // acc_par: parity bit per buffer
-    uint32_t local = 0;
+    const uint64_t adesc0 = smem_desc(sbase + OFF_A, 0, 1024, kSwizzle128B);
+    const uint64_t bdesc0 = smem_desc(sbase + OFF_B, 0, 1024, kSwizzle128B);
+    uint32_t stage = 0, phase = 0, acc_par = 0, local = 0;
+    uint32_t slot = 0, slot_phase = 0;
     bool ok = true;
     for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
       const uint32_t buf = local & 1u;
-      const uint32_t n0 = (tile / p.num_m_tiles) * BN;
-      const uint32_t sfb_shift = 4u + (n0 % 128) / 32;       // B scales start 4 columns into a slot
+      // This accumulator was drained (tile - 2), and the columns it shares with
+      // the other accumulator were read for the previous tile.
       if (!(ok = warp_mbar_wait(bar_acc_empty + 8 * buf, ((acc_par >> buf) & 1u) ^ 1u))) break;
       acc_par ^= 1u << buf;
+      if (local > 0 && !(ok = warp_mbar_wait(bar_overlap, (local - 1) & 1u))) break;
       tc_fence_after();
-      const uint32_t d_tmem = tmem_base + buf * BN;
+      const uint32_t d_tmem = tmem_base + acc_col(buf);
       for (uint32_t ks = 0; ks < p.num_k_stages; ++ks) {
         if (!(ok = warp_mbar_wait(bar_full + 8 * stage, phase))) break;
+        if (!(ok = warp_mbar_wait(bar_sf_full + 8 * slot, slot_phase))) break;
         tc_fence_after();
         if (lane == 0) {
           const uint64_t ad = adesc0 + stage * (A_BYTES >> 4);
-          const uint64_t bd = bdesc0 + stage * (C::B_BYTES >> 4);
-          const uint64_t sad = sfadesc0 + stage * (SFA_BYTES >> 4);
-          const uint64_t sbd = sfbdesc0 + stage * (SFB_BYTES >> 4);
+          const uint64_t bd = bdesc0 + stage * (B_BYTES >> 4);
+          const uint32_t sf = tmem_base + SF_COL0 + SF_SLOT_COLS * slot;
           const uint32_t natoms = min(4u, p.k_atoms - 4 * ks);
-          // B-scale atoms past the last row tile are not loaded; their slot
-          // columns then hold stale values that only reach output columns >= N.
-          if (natoms == 4) {
-#pragma unroll
-            for (uint32_t j = 0; j < 4; ++j) {
-              tc_cp_32x128b_warpx4(sf, sad + 32 * j);                  // 512-byte atoms: 32 x 16 B
-              tc_cp_32x128b_warpx4(sf + 4, sbd + 32 * j);
-              tc_cp_32x128b_warpx4(sf + 8, sbd + 128 + 32 * j);       // second atom, 2048 B further
-              tc_mma_nvf4(d_tmem, ad + 2 * j, bd + 2 * j, C::IDESC, sf, sf + sfb_shift, (ks | j) != 0u);
-              sf += SF_SLOT_COLS;
-              if (sf == sf_end) sf = sf_begin;
-            }
-          } else {
-            for (uint32_t j = 0; j < natoms; ++j) {
-              tc_cp_32x128b_warpx4(sf, sad + 32 * j);
-              tc_cp_32x128b_warpx4(sf + 4, sbd + 32 * j);
-              tc_cp_32x128b_warpx4(sf + 8, sbd + 128 + 32 * j);
-              tc_mma_nvf4(d_tmem, ad + 2 * j, bd + 2 * j, C::IDESC, sf, sf + sfb_shift, (ks | j) != 0u);
-              sf += SF_SLOT_COLS;
-              if (sf == sf_end) sf = sf_begin;
-            }
-          }
+          for (uint32_t j = 0; j < natoms; ++j)     // 32 bytes (64 FP4 elements) per k step
+            tc_mma_nvf4(d_tmem, ad + 2 * j, bd + 2 * j, IDESC, sf + 4 * j, sf + 16 + 8 * j, (ks | j) != 0u);
           tc_commit(bar_empty + 8 * stage);
+          tc_commit(bar_sf_free + 8 * slot);
         }
         __syncwarp();
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        if (++slot == SF_SLOTS) { slot = 0; slot_phase ^= 1; }
       }
       if (!ok) break;
       if (lane == 0) tc_commit(bar_acc_full + 8 * buf);
@@ -225,67 +209,104 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       mbar_wait_drain(bar_drain, 0, 200000000ull);
     }
     __syncwarp();
+  } else if (warp >= 2 + EPI_WARPS) {
+    // ------------------------------------------------------------ scale writers
+    const uint32_t q = warp & 3u;                             // TMEM sub-partition of this warp
+    const uint32_t lane_base = (q * 32u) << 16;
+    uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0;
+    bool ok = true;
+    for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (uint32_t ks = 0; ks < p.num_k_stages; ++ks) {
+        if (!(ok = warp_mbar_wait(bar_sf_free + 8 * slot, slot_phase ^ 1))) break;   // MMAs two stages back done
+        if (!(ok = warp_mbar_wait(bar_full + 8 * stage, phase))) break;
+        tc_fence_after();
+        const uint8_t* sfa = smem + OFF_SFA + stage * SFA_BYTES + 16 * lane;
+        const uint8_t* sfb = smem + OFF_SFB + stage * SFB_BYTES + 16 * lane;
+        const uint32_t col = lane_base + tmem_base + SF_COL0 + SF_SLOT_COLS * slot;
+        const uint32_t natoms = min(4u, p.k_atoms - 4 * ks);
+        for (uint32_t j = 0; j < natoms; ++j) {
+          // Atom row `lane` holds rows lane, lane+32, lane+64, lane+96 (4 bytes each);
+          // column c gets rows 32c + lane, as tcgen05.cp .32x128b.warpx4 would place them.
+          const uint4 a = *reinterpret_cast<const uint4*>(sfa + 512 * j);
+          const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j);
+          const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + 2048 + 512 * j);
+          const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+          const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+          tc_st_32x32b_x4(col + 4 * j, aw);
+          tc_st_32x32b_x8(col + 16 + 8 * j, bw);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_sf_full + 8 * slot);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        if (++slot == SF_SLOTS) { slot = 0; slot_phase ^= 1; }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
-    const uint32_t q = warp & 3u;                            // TMEM sub-partition of this warp
-    const uint32_t row = q * 32 + lane;                      // row of the tile held by this thread
-    const bool issuer = (warp == 2 && lane == 0);
+    const uint32_t q = warp & 3u;                             // TMEM sub-partition of this warp
+    const uint32_t h = (warp - 2) >> 2;                       // which 64-column chunk of each pair
+    const uint32_t row = q * 32 + lane;                       // row of the tile held by this thread
     const float alpha = __ldg(p.t_x) * __ldg(p.t_w);
-    uint32_t acc_par = 0;                                    // parity bit per accumulator buffer
-    uint32_t chunk_count = 0, local = 0;
-    bool dead = false;                                       // a wait ran out: keep the barrier
-    for (uint32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {  // sequence, skip work
+    uint8_t* cbuf = smem + OFF_C + (warp - 2) * C_BYTES;      // this warp's 32 x 128 B staging
+    const uint32_t cbuf_s = smem_addr(cbuf);
+    uint32_t acc_par = 0, local = 0;
+    bool dead = false;                                        // a wait ran out: skip work
+    for (uint32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const uint32_t mt = tile % p.num_m_tiles, nt = tile / p.num_m_tiles;
       const uint32_t buf = local & 1u;
       if (!dead && !warp_mbar_wait(bar_acc_full + 8 * buf, (acc_par >> buf) & 1u)) dead = true;
       acc_par ^= 1u << buf;
+      if (dead) continue;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((q * 32u) << 16) + buf * BN;
-      uint32_t v[32];
-      if (!dead) tc_ld_32x32b_x32(taddr, v);
+      const uint32_t taddr = tmem_base + ((q * 32u) << 16) + acc_col(buf);
+      // Chunk (64 columns) in the region shared with the other accumulator first:
+      // chunks 2, 3 of accumulator 0 and 0, 1 of accumulator 1.
+      const uint32_t ch_first = (buf ? 0u : 2u) + h, ch_second = (buf ? 2u : 0u) + h;
+      uint32_t v[64];
+      tc_ld_32x32b_x64(taddr + ch_first * C_COLS, v);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_overlap);
 #pragma unroll 1
-      for (int ch = 0; ch < BN / C_COLS; ++ch) {
-        uint32_t packed[16];
-        if (!dead) {
-          tc_wait_ld();
+      for (int part = 0; part < 2; ++part) {
+        const uint32_t ch = part ? ch_second : ch_first;
+        uint32_t packed[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float lo = __uint_as_float(v[2 * i]) * alpha, hi = __uint_as_float(v[2 * i + 1]) * alpha;
-            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(packed[i]) : "f"(hi), "f"(lo));
-          }
-          if (ch + 1 < BN / C_COLS) {
-            tc_ld_32x32b_x32(taddr + (uint32_t)(ch + 1) * C_COLS, v);   // next chunk in flight
-          } else {
-            tc_fence_before();                               // all TMEM reads of this tile issued
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_acc_empty + 8 * buf);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) packed[i] = 0u;
+        for (int e = 0; e < 32; ++e) {
+          const float lo = __uint_as_float(v[2 * e]) * alpha, hi = __uint_as_float(v[2 * e + 1]) * alpha;
+          asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(packed[e]) : "f"(hi), "f"(lo));
         }
-        const uint32_t col0 = nt * BN + ch * C_COLS;
-        const uint32_t cb = chunk_count & 1u;
-        if (issuer) bulk_wait_read<1>();
-        named_barrier_sync(1, 128);
-        uint8_t* cbuf = smem + C::OFF_C + cb * C_BYTES;
+        if (part == 0) tc_ld_32x32b_x64(taddr + ch_second * C_COLS, v);   // in flight during the store
+        if (lane == 0) bulk_wait_read<0>();                     // previous store done reading staging
+        __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          // 64-byte swizzle: 16-byte chunk i of row r sits at chunk i ^ ((r >> 1) & 3).
-          const uint32_t sw = ((uint32_t)i ^ ((row >> 1) & 3u)) * 16u;
-          *reinterpret_cast<uint4*>(cbuf + row * 64u + sw) =
-              make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        for (int e = 0; e < 8; ++e) {
+          // 128-byte swizzle: 16-byte chunk e of row r sits at chunk e ^ (r & 7).
+          const uint32_t sw = ((uint32_t)e ^ (lane & 7u)) * 16u;
+          *reinterpret_cast<uint4*>(cbuf + lane * 128u + sw) =
+              make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
         }
         fence_proxy_async_smem();
-        named_barrier_sync(1, 128);
-        if (issuer && !dead && col0 < p.N) {
-          tma_store_2d(&tmap_y, sbase + C::OFF_C + cb * C_BYTES, (int)col0, (int)(mt * BM));
+        __syncwarp();
+        const uint32_t col0 = nt * BN + ch * C_COLS;
+        if (lane == 0 && col0 < p.N) {
+          tma_store_2d(&tmap_y, cbuf_s, (int)col0, (int)(mt * BM + q * 32));
           bulk_commit();
         }
-        ++chunk_count;
+        if (part == 0) {
+          tc_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_acc_empty + 8 * buf);   // all of this tile's TMEM read
+        }
       }
     }
-    if (issuer) bulk_wait<0>();
+    if (lane == 0) bulk_wait<0>();
+    __syncwarp();
+    (void)row;
   }
 
   tc_fence_before();

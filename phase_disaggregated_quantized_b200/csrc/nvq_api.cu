@@ -275,19 +275,17 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const flo
 
 namespace {
 
-template <int BN>
 nvq_status launch_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const float* t_x, const uint8_t* w_codes,
                        const uint8_t* w_scales, const float* t_w, void* y_bf16, int64_t M, int64_t N, int64_t K,
                        cudaStream_t stream) {
   using namespace nvq::w4a4;
-  using C = Cfg<BN>;
   CUtensorMap ma, mb, my;
   if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
                    BKB, BM) ||
       !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
                    BKB, BN) ||
       !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2,
-                   C_COLS, BM, CU_TENSOR_MAP_SWIZZLE_64B))
+                   C_COLS, 32))                               // one epilogue warp: 32 rows x 64 columns
     return fail(NVQ_ERR_CUDA, "nvfp4_gemm_w4a4: tensor map encoding failed");
   Params p;
   p.x_scales = x_scales;
@@ -305,13 +303,12 @@ nvq_status launch_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const fl
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(nvfp4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    C::SMEM_BYTES);
+    attr_err = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "nvfp4_gemm_w4a4: smem attribute");
   const uint64_t tiles = (uint64_t)p.num_m_tiles * p.num_n_tiles;
   const int grid = (int)std::min<uint64_t>(tiles, (uint64_t)sm_count());
-  nvfp4_gemm_kernel<BN><<<grid, THREADS, C::SMEM_BYTES, stream>>>(ma, mb, my, p);
+  nvfp4_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, my, p);
   return launch_status("nvfp4_gemm_kernel");
 }
 
@@ -332,10 +329,7 @@ nvq_status nvfp4_gemm_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, cons
       !aligned16(y_bf16) || (reinterpret_cast<uintptr_t>(t_x) & 3u) || (reinterpret_cast<uintptr_t>(t_w) & 3u))
     return fail(NVQ_ERR_MISALIGNED, "nvfp4_gemm_w4a4: pointer not aligned");
   if (M == 0) return NVQ_OK;
-  // 192-wide N tiles: two accumulators (384 TMEM columns) fit beside the scales,
-  // and every tile starts at a row offset that is a multiple of 64 within its
-  // 128-row scale atom, so the B-scale TMEM address moves by 0 or 2 columns.
-  return launch_w4a4<192>(x_codes, x_scales, t_x, w_codes, w_scales, t_w, y_bf16, M, N, K, stream);
+  return launch_w4a4(x_codes, x_scales, t_x, w_codes, w_scales, t_w, y_bf16, M, N, K, stream);
 }
 
 // ------------------------------------------------------------------ INT4
