@@ -5,8 +5,11 @@
   python -m phase_disaggregated_quantized_b200.profile_case --op quantize --M 8192 --K 12288
 
 Inputs are drawn on the GPU from the seeded generators; the offline steps
-(weight quantization and reorder) run once before the measured calls.  Prints
-the mean CUDA-event time per call of the measured op.
+(weight quantization and reorder) run once before the measured calls.  The
+measured calls are captured in a CUDA graph and replayed once; prints the
+mean CUDA-event time per call.  Inputs stay the same between calls, so small
+weights can be served from L2 unless ``--copies`` cycles through more weight
+bytes than L2 holds (126 MB).
 """
 from __future__ import annotations
 
@@ -25,6 +28,8 @@ def main():
     ap.add_argument("--K", type=int, required=True)
     ap.add_argument("--N", type=int, default=0)
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--copies", type=int, default=1,
+                    help="w4a16: cycle through this many weight copies (a total above L2 gives cold-cache reads)")
     a = ap.parse_args()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -40,10 +45,15 @@ def main():
     elif a.op == "w4a16":
         w = synth.weights_cuda(a.N, a.K, seed=11, device=dev)
         codes, scales = nvq.int4_quantize(w)
-        pc, ps = nvq.int4_pack_weights(codes, scales, a.N, a.K)
+        packed = [nvq.int4_pack_weights(codes, scales, a.N, a.K) for _ in range(a.copies)]
         y = torch.empty(a.M, a.N, dtype=torch.bfloat16, device=dev)
         ws = torch.empty(max(16, nvq.w4a16_workspace_bytes(a.M, a.N, a.K)), dtype=torch.uint8, device=dev)
-        run = lambda: nvq.w4a16_gemm(x, pc, ps, a.N, y=y, workspace=ws)  # noqa: E731
+        calls = [0]
+
+        def run():
+            pc, ps = packed[calls[0] % len(packed)]
+            calls[0] += 1
+            nvq.w4a16_gemm(x, pc, ps, a.N, y=y, workspace=ws)
         work = a.N * a.K / 2 + 2 * a.N * a.K / 128 + 2 * a.M * a.K + 2 * a.M * a.N
         unit = "GB/s"
     else:
@@ -54,13 +64,22 @@ def main():
         run = lambda: nvq.nvfp4_quantize(x, None, codes=codes, scales=sc, tensor_scale_out=t, workspace=ws)  # noqa
         work = 2.0 * a.M * a.K * 2 + a.M * a.K * (0.5 + 1 / 16)
         unit = "GB/s"
-    run()
+    run()                                   # first call sets kernel attributes
+    torch.cuda.synchronize()
+    # Time a captured graph of `iters` calls: no host launch overhead between them.
+    stream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(graph, stream=stream):
+            for _ in range(a.iters):
+                run()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(a.iters):
-        run()
-    e1.record()
+    with torch.cuda.stream(stream):
+        graph.replay()                      # warm
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
     torch.cuda.synchronize()
     nvq.check_device_error()
     s = e0.elapsed_time(e1) / 1e3 / a.iters
