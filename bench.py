@@ -270,14 +270,14 @@ def run_gpu(args):
             wsb = nvq.w4a16_workspace_bytes(M, N, K)
             dec.append(dict(M=M, K=K, N=N, layer=i, x=x, pc=dec_w[mi][i][0], ps=dec_w[mi][i][1],
                             y=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
-                            ws=torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev), split=wsb > 0))
+                            ws=torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)))
     torch.cuda.synchronize()
 
     # external=True: the records become timestamp nodes of the captured graph
     ev = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
     q_ev = [(ev(), ev()) for _ in pre]
     g_ev = [(ev(), ev()) for _ in pre]
-    d_ev = [(ev(), ev()) for _ in dec]
+    d_ev = [(ev(), ev()) for _ in DECODE_BATCHES]     # one timed region per batch size
     pre_ev = (ev(), ev())
 
     def step():
@@ -292,12 +292,14 @@ def run_gpu(args):
                                 stream=stream)
             gb.record(stream)
         pre_ev[1].record(stream)
-        for D, (da, db) in zip(dec, d_ev):
+        for M, (da, db) in zip(DECODE_BATCHES, d_ev):
             da.record(stream)
-            nvq.w4a16_gemm(D["x"], D["pc"], D["ps"], D["N"], y=D["y"], workspace=D["ws"], stream=stream)
+            for D in dec:
+                if D["M"] == M:
+                    nvq.w4a16_gemm(D["x"], D["pc"], D["ps"], D["N"], y=D["y"], workspace=D["ws"], stream=stream)
             db.record(stream)
 
-    launches_per_step = 3 * len(pre) + sum(2 if D["split"] else 1 for D in dec)
+    launches_per_step = 3 * len(pre) + len(dec)
     step()                                  # first calls set kernel attributes outside capture
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
@@ -313,7 +315,7 @@ def run_gpu(args):
     t_start, t_end = ev(), ev()
     q_ms = [0.0] * len(pre)
     g_ms = [0.0] * len(pre)
-    d_ms = [0.0] * len(dec)
+    d_ms = [0.0] * len(DECODE_BATCHES)
     pre_ms = 0.0
     if world > 1:
         dist.barrier()
@@ -327,7 +329,7 @@ def run_gpu(args):
             for j in range(len(pre)):
                 q_ms[j] += q_ev[j][0].elapsed_time(q_ev[j][1])
                 g_ms[j] += g_ev[j][0].elapsed_time(g_ev[j][1])
-            for j in range(len(dec)):
+            for j in range(len(DECODE_BATCHES)):
                 d_ms[j] += d_ev[j][0].elapsed_time(d_ev[j][1])
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -347,14 +349,15 @@ def run_gpu(args):
         return N * K / 2 + 2 * N * K / 128 + 2 * M * K + 2 * M * N
 
     per_batch = {}
-    for M in DECODE_BATCHES:
+    dec_b = dec_s = 0.0
+    for mi, M in enumerate(DECODE_BATCHES):
         js = [j for j, D in enumerate(dec) if D["M"] == M]
         b = sum(dec_bytes(dec[j]) for j in js)
-        s = sum(d_ms[j] for j in js) / 1e3 / K_steps
+        s = d_ms[mi] / 1e3 / K_steps
         per_batch[str(M)] = {"GB/s": b / s / 1e9, "us_per_call": 1e6 * s / len(js)}
-    small = [j for j, D in enumerate(dec) if D["M"] <= 16]
-    dec_b = sum(dec_bytes(dec[j]) for j in small)
-    dec_s = sum(d_ms[j] for j in small) / 1e3 / K_steps
+        if M <= 16:
+            dec_b += b
+            dec_s += s
 
     peaks, peaks_kind = load_peaks()
     fp4_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP4_OVER_BF16
@@ -455,12 +458,15 @@ def measure_e2e(torch, nvq, pre, stream, steps: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 400 on the GPU, about one second; 20 for the CPU oracle arm)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="nvq", choices=("nvq", "reference"))
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.steps is None:
+        args.steps = 20 if args.impl == "reference" else 400
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)

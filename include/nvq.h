@@ -155,9 +155,10 @@ nvq_status int4_quantize(const void* w_bf16, int64_t N, int64_t K, uint8_t* code
 
 /* ------------------------------------------------------------------------ *
  * Offline reorder of INT4 codes and group scales into the decode kernel's
- * fragment order (MARLIN page, "weight layout": codes and scales are permuted
- * ahead of time so each thread's loads are regular and dequantize straight
- * into tensor-core fragment order).  A bijection: no byte is added or lost.
+ * fragment order (MARLIN page, abeam.tech, the section on the offline weight
+ * reorder: codes and scales are permuted ahead of time so each thread's loads
+ * are regular and dequantize straight into tensor-core fragment order).  A
+ * bijection: no byte is added or lost.
  *
  * Unit = 16 weight rows x one 128-wide group: 1024 code bytes at unit index
  * (n/16)*(K/128) + k/128.  Inside a unit, 32-bit word 128h + 4lane + jj (h in
@@ -176,18 +177,23 @@ nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int6
                              uint8_t* packed_codes, void* packed_scales, void* stream);
 
 /* ------------------------------------------------------------------------ *
- * W4A16 decode GEMM (MARLIN page: FP16/BF16 activations x INT4 weights with
- * group-128 scales, streaming the weights asynchronously with an L2-sparing
- * cache policy, dequantizing in registers next to the tensor-core MMAs).
+ * W4A16 decode GEMM (MARLIN page, abeam.tech: FP16/BF16 activations x INT4
+ * weights with group-128 scales, streaming the weights asynchronously with an
+ * L2-sparing cache policy, dequantizing in registers next to the tensor-core
+ * MMAs, several warps sharing one output tile).
  *
  *   Y[m, n] = bf16_RNE( sum_g s[n, g] * sum_{k in g} x[m, k] * (u[n, k] - 8) )
- * with the inner sums accumulated in FP32 (the products x * (u - 8) are exact)
- * and the group scale applied in FP32.
+ * with the inner sums accumulated in FP32 by the tensor cores and the group
+ * scale applied in FP32.  All products are exact; for M <= 8 the inner sum is
+ * formed as sum x * (128 + u) + sum x * (-136), equal up to FP32 rounding.
+ * Group sums are added in an order fixed by the shapes and the GPU's SM count,
+ * so repeated calls give identical results.
  *
  * x_bf16 [M, K] BF16; packed_codes / packed_scales from int4_pack_weights;
  * y_bf16 [M, N] BF16, row stride N, written.
- * workspace: w4a16_workspace_bytes(M, N, K) bytes of device scratch (split-K
- * partial sums); may be NULL when that is 0.
+ * workspace / workspace_bytes: unused (w4a16_workspace_bytes returns 0, the
+ * partial sums stay on chip); kept so callers need not change.
+ * Runs best for M <= 16; larger M is processed 32 rows per pass over W.
  * Shape rules: M >= 0, N % 16 == 0, K % 128 == 0.
  * ------------------------------------------------------------------------ */
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);

@@ -79,51 +79,49 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uin
 
 constexpr int64_t kMaxDim = (int64_t)1 << 31;
 
-// Decode work split: KS warps of a CTA share a 16-row tile (in-CTA K split, no
-// workspace); a global K split (FP32 partials + reduce kernel) only when the
-// weight matrix is too small to give ~1024 warps otherwise.
-struct W4a16Plan {
-  int nt8;          // batch tiles of 8 rows per pass
-  int ks;           // warps per row tile
-  uint32_t splits;  // global K splits
-};
-
-W4a16Plan w4a16_plan(int64_t M, int64_t N, int64_t K) {
-  W4a16Plan pl;
-  pl.nt8 = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
-  const uint32_t G = (uint32_t)(K / 128);
-  const uint64_t tiles = (uint64_t)(N / 16);
-  const uint64_t want = 1024;
-  pl.ks = 1;
-  while (pl.ks < 4 && tiles * pl.ks < want && G % (2 * pl.ks) == 0) pl.ks *= 2;
-  pl.splits = 1;
-  if (M <= 64) {
-    while (tiles * pl.ks * pl.splits < want && G % (pl.ks * pl.splits * 2) == 0 && pl.splits < 16) pl.splits *= 2;
-  }
-  return pl;
-}
-
-template <int NT8, int KS>
-nvq_status launch_w4a16_t(const void* x, const uint8_t* pc, const void* ps, void* y, float* ws, int64_t M,
-                          int64_t N, int64_t K, uint32_t splits, cudaStream_t stream) {
-  using namespace nvq::w4a16;
-  const uint32_t G = (uint32_t)(K / 128);
-  const uint32_t gps = G / splits;
-  constexpr int RT = WARPS / KS;
-  const uint64_t cta_rows = (uint64_t)((N / 16 + RT - 1) / RT);
-  const uint64_t grid = cta_rows * splits;
-  w4a16_kernel<NT8, KS><<<(unsigned)grid, THREADS, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(x), reinterpret_cast<const uint4*>(pc), static_cast<const uint32_t*>(ps),
-      static_cast<__nv_bfloat16*>(y), ws, (uint32_t)M, (uint32_t)N, (uint32_t)K, gps, splits);
-  return launch_status("w4a16_kernel");
-}
+// Decode launch: a persistent grid of clusters of nvq::w4a16::CS CTAs, as many
+// as can be resident at once (one CTA per SM), never more clusters than 16-row
+// tiles.  Batch rows are handled 8 * NT8 at a time.
+constexpr int kMaxDevices = 64;
 
 template <int NT8>
-nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* y, float* ws, int64_t M, int64_t N,
-                        int64_t K, const W4a16Plan& pl, cudaStream_t stream) {
-  if (pl.ks == 4) return launch_w4a16_t<NT8, 4>(x, pc, ps, y, ws, M, N, K, pl.splits, stream);
-  if (pl.ks == 2) return launch_w4a16_t<NT8, 2>(x, pc, ps, y, ws, M, N, K, pl.splits, stream);
-  return launch_w4a16_t<NT8, 1>(x, pc, ps, y, ws, M, N, K, pl.splits, stream);
+nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* y, int64_t M, int64_t N, int64_t K,
+                        cudaStream_t stream) {
+  using C = nvq::w4a16::Cfg<NT8>;
+  auto fn = nvq::w4a16::w4a16_kernel<NT8>;
+  static int max_clusters[kMaxDevices] = {};     // 0: not queried yet on that device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(NVQ_ERR_CUDA, "w4a16_gemm: device index out of range");
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nvq::w4a16::CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (max_clusters[dev] == 0) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm: shared memory attribute");
+    cfg.gridDim = dim3(nvq::w4a16::CS, 1, 1);
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, fn, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm: cudaOccupancyMaxActiveClusters");
+    if (n < 1) return fail(NVQ_ERR_CUDA, "w4a16_gemm: no cluster of the decode kernel fits on this GPU");
+    max_clusters[dev] = n;
+  }
+  const int64_t tiles = N / 16;
+  const int64_t nclu = std::min<int64_t>(max_clusters[dev], tiles);
+  cfg.gridDim = dim3((unsigned)(nclu * nvq::w4a16::CS), 1, 1);
+  e = cudaLaunchKernelEx(&cfg, fn, static_cast<const __nv_bfloat16*>(x), pc, static_cast<const uint8_t*>(ps),
+                         static_cast<__nv_bfloat16*>(y), (uint32_t)M, (uint32_t)N, (uint32_t)K);
+  if (e != cudaSuccess) return cuda_fail(e, "w4a16_kernel launch");
+  return launch_status("w4a16_kernel");
 }
 
 }  // namespace
@@ -374,39 +372,28 @@ nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int6
 
 // ------------------------------------------------------------------ W4A16 decode GEMM
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  if (M <= 0 || N <= 0 || K <= 0 || N % 16 || K % 128) return 0;
-  const W4a16Plan pl = w4a16_plan(M, N, K);
-  return pl.splits <= 1 ? 0 : (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(float);
+  (void)M;
+  (void)N;
+  (void)K;
+  return 0;                                      // partial sums stay on chip
 }
 
 nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const void* packed_scales, void* y_bf16,
                       int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes, void* stream_) {
+  (void)workspace;
+  (void)workspace_bytes;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "w4a16_gemm: bad sizes");
   if (N % 16 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_gemm: need N % 16 == 0, K % 128 == 0");
-  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_gemm: too large");
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || (N / 16) * (K / 128) >= ((int64_t)1 << 32))
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_gemm: too large");
   if (M == 0) return NVQ_OK;
   if (!x_bf16 || !packed_codes || !packed_scales || !y_bf16) return fail(NVQ_ERR_INVALID_ARG, "w4a16_gemm: NULL pointer");
   if (!aligned16(x_bf16) || !aligned16(packed_codes) || !aligned16(packed_scales) || !aligned16(y_bf16))
     return fail(NVQ_ERR_MISALIGNED, "w4a16_gemm: pointer not 16-byte aligned");
-  const W4a16Plan pl = w4a16_plan(M, N, K);
-  float* ws = nullptr;
-  if (pl.splits > 1) {
-    const size_t need = (size_t)pl.splits * (size_t)M * (size_t)N * sizeof(float);
-    if (workspace == nullptr || workspace_bytes < need) return fail(NVQ_ERR_WORKSPACE, "w4a16_gemm: workspace too small");
-    if (!aligned16(workspace)) return fail(NVQ_ERR_MISALIGNED, "w4a16_gemm: workspace not 16-byte aligned");
-    ws = static_cast<float*>(workspace);
-  }
-  nvq_status st;
-  if (pl.nt8 == 1) st = launch_w4a16<1>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, pl, stream);
-  else if (pl.nt8 == 2) st = launch_w4a16<2>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, pl, stream);
-  else st = launch_w4a16<4>(x_bf16, packed_codes, packed_scales, y_bf16, ws, M, N, K, pl, stream);
-  if (st != NVQ_OK || pl.splits == 1) return st;
-  const uint64_t n4 = (uint64_t)M * (uint64_t)N / 4;
-  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>((n4 + 255) / 256, (uint64_t)sm_count() * 8));
-  nvq::w4a16::w4a16_reduce_kernel<<<grid, 256, 0, stream>>>(static_cast<const float4*>(workspace),
-                                                            static_cast<uint2*>(y_bf16), pl.splits, n4);
-  return launch_status("w4a16_reduce_kernel");
+  if (M <= 8) return launch_w4a16<1>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
+  if (M <= 16) return launch_w4a16<2>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
+  return launch_w4a16<4>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
 }
 
 }  // extern "C"

@@ -39,8 +39,9 @@ def test_size_helpers(L):
     assert L.nvfp4_scales_bytes(10, 100) == 0          # K % 64 != 0
     assert L.nvfp4_quantize_workspace_bytes(0, 64) == 0
     assert L.nvfp4_quantize_workspace_bytes(128, 512) > 0
-    assert L.w4a16_workspace_bytes(1, 4096, 4096) == 0          # in-CTA K split suffices
-    assert L.w4a16_workspace_bytes(4096, 4096, 4096) == 0   # no split at large batch
+    assert L.w4a16_workspace_bytes(1, 4096, 4096) == 0          # partial sums stay on chip
+    assert L.w4a16_workspace_bytes(4, 256, 4096) == 0
+    assert L.w4a16_workspace_bytes(4096, 4096, 4096) == 0
 
 
 FAKE = 0x7F0000000000          # 16-byte aligned, never dereferenced: validation fails first
@@ -82,9 +83,8 @@ def test_int4_calls_reject_bad_arguments(L):
     assert L.int4_pack_weights(_vp(ODD), _vp(FAKE), 32, 128, _vp(FAKE), _vp(FAKE), None) == 3
     w = L.w4a16_gemm
     assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 24, 128, None, 0, None) == 2
-    assert L.w4a16_workspace_bytes(4, 256, 4096) > 0                                        # small N: global split
-    assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 256, 4096, None, 0, None) == 4    # split-K workspace
-    assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(ODD), 4, 256, 4096, _vp(FAKE), 1 << 30, None) == 3
+    assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(ODD), 4, 256, 4096, None, 0, None) == 3    # y misaligned
+    assert w(_vp(FAKE), _vp(FAKE), None, _vp(FAKE), 4, 256, 4096, None, 0, None) == 1         # NULL scales
 
 
 def test_zero_sized_calls_are_noops(L):
