@@ -39,6 +39,26 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP4_OVER_BF16 = 4.0     # nominal dense ratio: 9 PF NVFP4 / 2.25 PF BF16
 
 
+def rank_seed(base: int, layer: int, rank: int) -> int:
+    """Seed of one layer's synthetic input on one rank: every rank draws its own
+    batch, so N ranks process N independent workloads (weak scaling)."""
+    return base + 10 * layer + 100000 * rank
+
+
+def max_over_ranks(torch, dist, values, device):
+    """Element-wise maximum of per-rank timings over the process group (the job
+    takes as long as its slowest rank); a no-op without a multi-rank group."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_rate(units_per_rank: float, world: int, seconds: float) -> float:
+    """Units processed by all ranks together per second of the slowest rank."""
+    return world * units_per_rank / seconds
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -240,7 +260,7 @@ def run_gpu(args):
     # ---------------- prefill buffers (weights quantized offline, untimed)
     pre = []
     for i, (name, K, N) in enumerate(LINEARS):
-        seed = 2000 + 10 * i + 100000 * rank
+        seed = rank_seed(2000, i, rank)
         x = synth.activations_cuda(PREFILL_M, K, seed, device=dev)
         w = synth.weights_cuda(N, K, seed, device=dev)
         wq = nvq.nvfp4_quantize(w)
@@ -266,7 +286,7 @@ def run_gpu(args):
     dec = []
     for mi, M in enumerate(DECODE_BATCHES):
         for i, (name, K, N) in enumerate(LINEARS):
-            x = synth.activations_cuda(M, K, 4000 + 10 * i + M + 100000 * rank, device=dev)
+            x = synth.activations_cuda(M, K, rank_seed(4000 + M, i, rank), device=dev)
             wsb = nvq.w4a16_workspace_bytes(M, N, K)
             dec.append(dict(M=M, K=K, N=N, layer=i, x=x, pc=dec_w[mi][i][0], ps=dec_w[mi][i][1],
                             y=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
@@ -363,23 +383,18 @@ def run_gpu(args):
     fp4_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP4_OVER_BF16
     fp4_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP4_OVER_BF16
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    gemm_tflops = gemm_flops / gemm_s / 1e12
-
     # max over ranks of the step time and of the per-kernel sums
-    vals = torch.tensor([total_ms, pre_s, gemm_s, dec_s], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, pre_s, gemm_s_max, dec_s_max = [float(v) for v in vals.cpu()]
-    value = world * gemm_flops / pre_s / 1e12
+    total_ms, pre_s, gemm_s, dec_s = max_over_ranks(torch, dist if world > 1 else None,
+                                                    [total_ms, pre_s, gemm_s, dec_s], dev)
+    gemm_tflops = gemm_flops / gemm_s / 1e12          # per GPU (slowest rank): the kernel's roofline
+    value = whole_job_rate(gemm_flops, world, pre_s) / 1e12
 
     # ---------------- end to end through the public API with host buffers
     e2e = None
     if rank == 0 or world > 1:
         e2e = measure_e2e(torch, nvq, pre, stream, steps=max(2, min(args.steps, 5)))
     if world > 1:
-        t = torch.tensor([e2e["seconds"]], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["seconds"] = float(t.item())
+        e2e["seconds"] = max_over_ranks(torch, dist, [e2e["seconds"]], dev)[0]
 
     if rank == 0:
         clk = clocks.summary()

@@ -81,7 +81,23 @@ struct Params {
   uint32_t num_m_tiles, num_n_tiles, num_k_stages;
   uint32_t k_atoms;        // K / 64: scale atoms per 128-row tile
   uint32_t n_row_atoms;    // padded N / 128
+  uint32_t m_fastest;      // 1: tile index runs over row blocks first (A re-read per wave)
 };
+
+// Tile order: the tiles in flight at once (one per SM) cover a band of tiles
+// that re-reads one operand every wave.  The host picks the smaller operand for
+// that role (A_fastest: row blocks fastest, all of A swept per wave), so the
+// swept operand stays in L2 next to the output stream and each byte of the
+// other operand is read from HBM once.
+__device__ __forceinline__ void tile_coords(uint32_t tile, const Params& p, uint32_t& mt, uint32_t& nt) {
+  if (p.m_fastest) {
+    mt = tile % p.num_m_tiles;
+    nt = tile / p.num_m_tiles;
+  } else {
+    nt = tile % p.num_n_tiles;
+    mt = tile / p.num_n_tiles;
+  }
+}
 
 __device__ __forceinline__ uint32_t acc_col(uint32_t buf) { return buf ? ACC1_COL : 0u; }
 
@@ -140,7 +156,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       uint32_t pending = 0, pending_parity = 0;               // per-stage bit masks
       bool ok = true;
       for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const uint32_t mt = tile % p.num_m_tiles, nt = tile / p.num_m_tiles;
+        uint32_t mt, nt;
+        tile_coords(tile, p, mt, nt);
         const uint32_t nb_atoms = min(2u, p.n_row_atoms - 2 * nt);
         for (uint32_t ks = 0; ks < p.num_k_stages; ++ks) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
@@ -254,7 +271,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     uint32_t acc_par = 0, local = 0;
     bool dead = false;                                        // a wait ran out: skip work
     for (uint32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-      const uint32_t mt = tile % p.num_m_tiles, nt = tile / p.num_m_tiles;
+      uint32_t mt, nt;
+      tile_coords(tile, p, mt, nt);
       const uint32_t buf = local & 1u;
       if (!dead && !warp_mbar_wait(bar_acc_full + 8 * buf, (acc_par >> buf) & 1u)) dead = true;
       acc_par ^= 1u << buf;

@@ -298,6 +298,8 @@ nvq_status launch_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const fl
   p.num_k_stages = (uint32_t)((K / 2 + BKB - 1) / BKB);
   p.k_atoms = (uint32_t)(K / 64);
   p.n_row_atoms = (uint32_t)((N + 127) / 128);
+  // Sweep the smaller operand every wave (it stays in L2), stream the larger once.
+  p.m_fastest = (uint64_t)M <= (uint64_t)N ? 1u : 0u;   // both operands have K/2 + K/16 bytes per row
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
