@@ -32,9 +32,7 @@ constexpr int kAmaxThreads = 512;
 constexpr int kAmaxMaxBlocks = 592;       // 4 per SM on 148 SMs
 constexpr int kQuantThreads = 256;
 
-__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
-  // For non-negative bf16 the bit patterns order like the values.
-  const uint32_t x = a & 0x7FFF7FFFu, y = b & 0x7FFF7FFFu;
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t x, uint32_t y) {   // inputs already >= 0
   uint32_t r;
   asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(y));
   return r;
@@ -50,18 +48,16 @@ __global__ void __launch_bounds__(kAmaxThreads) nvfp4_amax_kernel(const uint4* _
   uint32_t m = 0;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  auto vmax = [](const uint4 v) {            // max |x| of 8 bf16, still packed in two halves
+    return bf16x2_max(bf16x2_max(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                      bf16x2_max(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  };
   for (; i + 3 * stride < nvec; i += 4 * stride) {
-    uint4 v0 = __ldg(x + i), v1 = __ldg(x + i + stride), v2 = __ldg(x + i + 2 * stride),
-          v3 = __ldg(x + i + 3 * stride);
-    m = bf16x2_absmax(m, bf16x2_absmax(bf16x2_absmax(v0.x, v0.y), bf16x2_absmax(v0.z, v0.w)));
-    m = bf16x2_absmax(m, bf16x2_absmax(bf16x2_absmax(v1.x, v1.y), bf16x2_absmax(v1.z, v1.w)));
-    m = bf16x2_absmax(m, bf16x2_absmax(bf16x2_absmax(v2.x, v2.y), bf16x2_absmax(v2.z, v2.w)));
-    m = bf16x2_absmax(m, bf16x2_absmax(bf16x2_absmax(v3.x, v3.y), bf16x2_absmax(v3.z, v3.w)));
+    const uint4 v0 = __ldg(x + i), v1 = __ldg(x + i + stride), v2 = __ldg(x + i + 2 * stride),
+                v3 = __ldg(x + i + 3 * stride);
+    m = bf16x2_max(m, bf16x2_max(bf16x2_max(vmax(v0), vmax(v1)), bf16x2_max(vmax(v2), vmax(v3))));
   }
-  for (; i < nvec; i += stride) {
-    uint4 v = __ldg(x + i);
-    m = bf16x2_absmax(m, bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w)));
-  }
+  for (; i < nvec; i += stride) m = bf16x2_max(m, vmax(__ldg(x + i)));
   float f = bf16x2_hmax_to_f32(m);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
@@ -101,20 +97,18 @@ __device__ __forceinline__ uint32_t e2m1x2_rn_satfinite(float hi, float lo) {
 
 __constant__ float c_e2m1_mid[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
 
-// amax_b > 6 mu t, or equal with the tie going up (upper code even)?
-__device__ __forceinline__ bool scale_passes(float amax, float mu, float t, uint32_t upper_code) {
-  const float r = __fmaf_rn(-__fmul_rn(mu, 6.0f), t, amax);   // exact sign
-  return r > 0.f || (r == 0.f && (upper_code & 1u) == 0u);
-}
-
 // E4M3_RNE_satfinite(amax / (6 t)) decided on the exact quotient.  The estimate
 // amax * fl(1/fl(6t)) is within ~2 ulp, so the answer is s0 or a neighbour.
-__device__ __forceinline__ uint32_t block_scale_code(float amax, float t, float inv6t) {
+// mid6[c] = 6 * (value(c) + value(c + 1)) / 2, exact in FP32 (at most 7
+// significant bits).
+__device__ __forceinline__ uint32_t block_scale_code(float amax, float t, float inv6t, const float* mid6) {
   uint32_t s = e4m3_rn_satfinite(__fmul_rn(amax, inv6t));
-  if (s < 126u && scale_passes(amax, 0.5f * (e4m3_value(s) + e4m3_value(s + 1)), t, s + 1))
-    s += 1;
-  else if (s > 0u && !scale_passes(amax, 0.5f * (e4m3_value(s - 1) + e4m3_value(s)), t, s))
-    s -= 1;
+  const float r_up = __fmaf_rn(-mid6[s], t, amax);                      // exact sign (s <= 126)
+  if (s < 126u && (r_up > 0.f || (r_up == 0.f && ((s + 1u) & 1u) == 0u))) return s + 1u;
+  if (s > 0u) {
+    const float r_dn = __fmaf_rn(-mid6[s - 1u], t, amax);
+    if (!(r_dn > 0.f || (r_dn == 0.f && (s & 1u) == 0u))) return s - 1u;
+  }
   return s;
 }
 
@@ -139,17 +133,26 @@ __device__ __forceinline__ uint32_t e2m1_fast_code(uint32_t bf16_bits, float inv
   return e2m1x2_rn_satfinite(0.f, __fmul_rn(v, inv_d)) & 0xFu;
 }
 
-// Packed codes for 4 bf16x2 words (8 elements) -> 32 bits, fast path.
+// Packed codes for 4 bf16x2 words (8 elements) -> 32 bits, fast path.  The
+// signed product goes straight into the conversion: fl(-a * r) = -fl(a * r) and
+// round-to-nearest-even is symmetric, so the code of -a is the code of a with
+// the sign bit set -- also for a product that rounds to zero (R6).
 __device__ __forceinline__ uint32_t codes8_fast(const uint32_t* w, float inv_d) {
-  uint32_t out = 0;
+  float v[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float alo = __uint_as_float((w[i] & 0x7FFFu) << 16);
-    const float ahi = __uint_as_float(w[i] & 0x7FFF0000u);
-    uint32_t byte = e2m1x2_rn_satfinite(__fmul_rn(ahi, inv_d), __fmul_rn(alo, inv_d));
-    byte |= ((w[i] >> 12) & 0x8u) | ((w[i] >> 24) & 0x80u);       // signs of x
-    out |= byte << (8 * i);
+    v[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), inv_d);            // even k (low half)
+    v[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv_d); // odd k (high half)
   }
+  uint32_t out;
+  asm("{ .reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3}; }"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
   return out;
 }
 
@@ -183,6 +186,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(
   __shared__ float s_inv_d[128];
   __shared__ uint32_t s_fast_ok[128];
   __shared__ uint4 s_thr[128];                               // 7 thresholds (bf16 bits) + pad
+  __shared__ float s_mid6[128];                              // 6 x midpoints between E4M3 codes
   __shared__ float s_t;
   if (threadIdx.x < 32) {
     float m = 0.f;
@@ -224,6 +228,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(
     }
     s_inv_d[c] = inv;
     s_fast_ok[c] = ok ? 1u : 0u;
+    s_mid6[c] = c < 126 ? __fmul_rn(6.0f, 0.5f * (S + e4m3_value(c + 1))) : 0.f;
     s_thr[c] = make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16), b[6] | (0x7F80u << 16));
   }
   __syncthreads();
@@ -234,6 +239,10 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(
   const uint32_t nblocks = rows * nbk;                       // < 2^32 (checked on the host)
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t stride = gridDim.x * blockDim.x;
+  // (row, block-in-row) of this thread's block, advanced without a division.
+  const uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t row = b0 / nbk, kb = b0 - row * nbk;
+  const uint32_t step_r = stride / nbk, step_kb = stride - step_r * nbk;
   for (uint32_t base = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); base < nblocks; base += stride) {
     const uint32_t b = base + lane;
     const bool valid = b < nblocks;                          // nblocks % 4 == 0: groups of 4 agree
@@ -243,10 +252,13 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(
       w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
       w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
     }
-    const uint32_t m2 = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(w[0], w[1]), bf16x2_absmax(w[2], w[3])),
-                                      bf16x2_absmax(bf16x2_absmax(w[4], w[5]), bf16x2_absmax(w[6], w[7])));
+    uint32_t a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = w[i] & 0x7FFF7FFFu;
+    const uint32_t m2 = bf16x2_max(bf16x2_max(bf16x2_max(a[0], a[1]), bf16x2_max(a[2], a[3])),
+                                   bf16x2_max(bf16x2_max(a[4], a[5]), bf16x2_max(a[6], a[7])));
     const float amax = bf16x2_hmax_to_f32(m2);
-    const uint32_t s = block_scale_code(amax, t, inv6t);
+    const uint32_t s = block_scale_code(amax, t, inv6t, s_mid6);
     uint2 c;
     if (s_fast_ok[s]) {
       const float inv_d = s_inv_d[s];
@@ -268,11 +280,16 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(
     if (valid) {
       codes[b] = c;
       if ((lane & 3u) == 0u) {
-        const uint32_t r = b / nbk, kb = b - r * nbk;
-        const size_t off = ((size_t)(r >> 7) * atoms_per_rowtile + (kb >> 2)) * 512u + (r & 31u) * 16u +
-                           ((r & 127u) >> 5) * 4u;
+        const size_t off = ((size_t)(row >> 7) * atoms_per_rowtile + (kb >> 2)) * 512u + (row & 31u) * 16u +
+                           ((row & 127u) >> 5) * 4u;
         *reinterpret_cast<uint32_t*>(scales + off) = sv;
       }
+    }
+    row += step_r;
+    kb += step_kb;
+    if (kb >= nbk) {
+      kb -= nbk;
+      ++row;
     }
   }
   // Zero the scales of the padding rows up to the next multiple of 128.
