@@ -85,6 +85,12 @@ def f32_rne(q: Fraction) -> float:
 def tensor_scale(x: np.ndarray) -> float:
     """Steps 1-2: t from the tensor's amax (readings R1, R2)."""
     amax = float(np.max(np.abs(x))) if x.size else 0.0
+    return tensor_scale_from_amax(amax)
+
+
+def tensor_scale_from_amax(amax: float) -> float:
+    """Step 2 alone, for callers that take max|x| of a tensor too large to hold
+    in float64: t = fp32_RN(amax / 2688), or 1 when amax = 0 (R1, R2)."""
     if amax == 0.0:
         return 1.0
     return f32_rne(Fraction(amax) / TENSOR_SCALE_DIVISOR)

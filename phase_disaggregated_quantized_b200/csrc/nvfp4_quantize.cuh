@@ -30,7 +30,7 @@ namespace nvq {
 
 constexpr int kAmaxThreads = 512;
 constexpr int kAmaxMaxBlocks = 592;       // 4 per SM on 148 SMs
-constexpr int kQuantThreads = 256;
+constexpr int kQuantThreads = 1024;   // two CTAs per SM: the per-CTA tables are built 296 times, not 1184
 
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t x, uint32_t y) {   // inputs already >= 0
   uint32_t r;
@@ -179,7 +179,7 @@ __device__ __forceinline__ uint32_t codes8_exact(const uint32_t* w, const uint32
 }
 
 // rows x K bf16 -> codes [rows, K/2], tiled scales, t.
-__global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(
+__global__ void __launch_bounds__(kQuantThreads, 2) nvfp4_quantize_kernel(
     const uint4* __restrict__ x, uint32_t rows, uint32_t K, const float* __restrict__ t_in,
     const float* __restrict__ partial, int npartial, uint2* __restrict__ codes,
     uint8_t* __restrict__ scales, float* __restrict__ t_out) {
@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(
   __shared__ uint32_t s_fast_ok[128];
   __shared__ uint4 s_thr[128];                               // 7 thresholds (bf16 bits) + pad
   __shared__ float s_mid6[128];                              // 6 x midpoints between E4M3 codes
+  __shared__ uint16_t s_b[127][8];                           // thresholds while the tables are built
   __shared__ float s_t;
   if (threadIdx.x < 32) {
     float m = 0.f;
@@ -206,12 +207,20 @@ __global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(
   // (fp32 quotient + cvt) provably agrees with them for every bf16 input: both
   // are monotone in |x|, so agreeing on both sides of every exact threshold
   // means agreeing everywhere.
+  // Thresholds first, one (code, midpoint) pair per thread ...
+  for (uint32_t i = threadIdx.x; i < 127u * 7u; i += blockDim.x) {
+    const uint32_t c = i / 7u, j = i - 7u * c;
+    s_b[c][j] = c == 0 ? (uint16_t)0x7F80u
+                       : (uint16_t)e2m1_threshold_bits(__fmul_rn(c_e2m1_mid[j], e4m3_value(c)), t, (int)j);
+  }
+  __syncthreads();
+  // ... then one thread per code checks the fast path against them.
   if (threadIdx.x < 127) {
     const uint32_t c = threadIdx.x;
     const float S = e4m3_value(c);
     uint32_t b[7];
 #pragma unroll
-    for (int i = 0; i < 7; ++i) b[i] = (c == 0) ? 0x7F80u : e2m1_threshold_bits(__fmul_rn(c_e2m1_mid[i], S), t, i);
+    for (int i = 0; i < 7; ++i) b[i] = s_b[c][i];
     const float d = __fmul_rn(S, t);
     const float inv = (c == 0) ? 0.f : __frcp_rn(d);
     bool ok = (c == 0) || (d >= 1.17549435e-38f && !isinf(inv));

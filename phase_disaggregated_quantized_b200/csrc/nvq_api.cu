@@ -218,7 +218,7 @@ nvq_status quantize_launch(const void* x_bf16, int64_t rows, int64_t K, const fl
   }
   const uint64_t nblocks = (uint64_t)rows * (uint64_t)(K / 16);
   const uint64_t want = (nblocks + nvq::kQuantThreads - 1) / nvq::kQuantThreads;
-  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count() * 8));
+  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count() * 2));
   nvq::nvfp4_quantize_kernel<<<grid, nvq::kQuantThreads, 0, stream>>>(
       static_cast<const uint4*>(x_bf16), (uint32_t)rows, (uint32_t)K, tensor_scale_in, partial, amax_blocks,
       reinterpret_cast<uint2*>(codes), scales, tensor_scale_out);
@@ -260,7 +260,7 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const flo
   }
   const uint64_t nblocks = (uint64_t)rows * (uint64_t)(K / 16);
   const uint64_t want = (nblocks + nvq::kQuantThreads - 1) / nvq::kQuantThreads;
-  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count() * 8));
+  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count() * 2));
   nvq::nvfp4_quantize_kernel<<<grid, nvq::kQuantThreads, 0, stream>>>(
       static_cast<const uint4*>(x_bf16), (uint32_t)rows, (uint32_t)K, tensor_scale_in,
       static_cast<const float*>(workspace), amax_blocks, reinterpret_cast<uint2*>(codes), scales,

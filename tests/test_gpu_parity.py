@@ -204,6 +204,39 @@ def test_gemm_qwen3_8b_prefill_full_size_sampled(layer):
     assert ok, (name, worst)
 
 
+@pytest.mark.parametrize("layer", range(4))
+def test_gemm_qwen3_32b_prefill_full_size_sampled(layer):
+    """M = 32768 on each Qwen3-32B linear (up to 1.7 GB of activations); sampled
+    rows and columns against the oracle.  Inputs are drawn on the GPU by the
+    seeded generators (a CPU draw of 0.8 G values would dominate the test); the
+    oracle receives them as bytes and takes max|x| of the whole tensor itself."""
+    name, K, N = synth.QWEN3_32B_LINEARS[layer]
+    M = 32768
+    x = synth.activations_cuda(M, K, seed=4000 + 10 * layer)
+    w = synth.weights_cuda(N, K, seed=4000 + 10 * layer)
+    gx = gpu_quant(x)
+    gw = gpu_quant(w)
+    y = nvq.nvfp4_gemm_w4a4(gx, gw, M, N, K)
+    nvq.check_device_error()
+    g = np.random.default_rng(100 + layer)
+    mi = np.sort(g.choice(M, 32, replace=False))
+    ni = np.sort(g.choice(N, 32, replace=False))
+    x_cpu, w_cpu = x.cpu(), w.cpu()
+    tx = onv.tensor_scale_from_amax(float(x_cpu.abs().max()))
+    tw = onv.tensor_scale_from_amax(float(w_cpu.abs().max()))
+    xc, xs, _ = onv.quantize(bf16_to_f64(x_cpu[torch.tensor(mi)]), t_in=tx)
+    wc, ws, _ = onv.quantize(bf16_to_f64(w_cpu[torch.tensor(ni)]), t_in=tw)
+    del x_cpu, w_cpu
+    assert float(gx[2].item()) == tx and float(gw[2].item()) == tw
+    np.testing.assert_array_equal(u8(gx[0])[mi], onv.pack_codes(xc))
+    np.testing.assert_array_equal(onv.scales_from_tiled(u8(gx[1]), M, K)[mi], xs)
+    np.testing.assert_array_equal(onv.scales_from_tiled(u8(gw[1]), N, K)[ni], ws)
+    y_ref = onv.gemm_ref(onv.dequantize(xc, xs, tx), onv.dequantize(wc, ws, tw))
+    y_s = bf16_to_f64(y[torch.tensor(mi).cuda()][:, torch.tensor(ni).cuda()])
+    ok, worst = onv.within_tolerance(y_s, y_ref)
+    assert ok, (name, worst)
+
+
 # ------------------------------------------------------------------ INT4 / W4A16
 
 def gpu_int4(w_cpu):
