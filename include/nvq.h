@@ -201,6 +201,37 @@ nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const voi
                       void* y_bf16, int64_t M, int64_t N, int64_t K,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------ *
+ * Phase dispatch over one master weight held in both formats (Disaggregated
+ * Quantization page, singularity-lens.com, the section on format
+ * disaggregation; Mix-Quant page, gist.science, section 2: NVFP4 W4A4 where
+ * the layer is compute-bound, weight-only INT4 where it streams weights):
+ *
+ *   M <= crossover_m:  Y = w4a16_gemm(X, packed INT4 W)
+ *   M >  crossover_m:  (codes, scales, t) = nvfp4_quantize(X), then
+ *                      Y = nvfp4_gemm_w4a4(X as NVFP4, NVFP4 W)
+ *
+ * Both weight forms come from the same BF16 master W [N, K]: w_codes /
+ * w_scales / w_t from nvfp4_quantize(W), w_packed_* from int4_quantize +
+ * int4_pack_weights.  Only the form the chosen path reads must be non-NULL.
+ * crossover_m < 0 selects nvq_default_crossover_m(): the largest M at which
+ * the W4A16 path was measured faster than quantize + W4A4 on B200 for the
+ * Qwen3-8B gate_up shape (K = 4096, N = 24576), weights read from HBM
+ * (python -m phase_disaggregated_quantized_b200.profile_case --op crossover).
+ * workspace: nvq_linear_workspace_bytes(M, N, K, crossover_m) bytes, 16-byte
+ * aligned (activation codes, scales, t and the quantizer's scratch), NULL when
+ * that is 0.  Output y_bf16 [M, N] BF16, row stride N.
+ * Shape rules: those of the chosen path (W4A16: N % 16 == 0, K % 128 == 0;
+ * W4A4: N % 8 == 0, K % 64 == 0).  Errors as the underlying calls.
+ * ------------------------------------------------------------------------ */
+int64_t nvq_default_crossover_m(void);
+size_t nvq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t crossover_m);
+nvq_status nvq_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K,
+                      const uint8_t* w_codes, const uint8_t* w_scales, const float* w_t,
+                      const uint8_t* w_packed_codes, const void* w_packed_scales,
+                      int64_t crossover_m, void* y_bf16, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -9,7 +9,9 @@ if the library or a GPU is missing, the calls raise.
 
 Prefill (Mix-Quant page, gist.science, section 2): ``nvfp4_quantize`` then
 ``nvfp4_gemm_w4a4``.  Decode (MARLIN page, abeam.tech): ``int4_quantize`` and
-``int4_pack_weights`` offline, then ``w4a16_gemm``.
+``int4_pack_weights`` offline, then ``w4a16_gemm``.  ``nvq_linear`` picks one
+of the two by the batch size M (Disaggregated Quantization page,
+singularity-lens.com: one master weight kept in both formats).
 """
 from __future__ import annotations
 
@@ -65,6 +67,9 @@ def lib() -> ctypes.CDLL:
             "int4_pack_weights": ([vp, vp, i64, i64, vp, vp, vp], i32),
             "w4a16_workspace_bytes": ([i64, i64, i64], sz),
             "w4a16_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp, sz, vp], i32),
+            "nvq_default_crossover_m": ([], i64),
+            "nvq_linear_workspace_bytes": ([i64, i64, i64, i64], sz),
+            "nvq_linear": ([vp, i64, i64, i64, vp, vp, vp, vp, vp, i64, vp, vp, sz, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -194,4 +199,38 @@ def w4a16_gemm(x, packed_codes, packed_scales, N: int, *, y=None, workspace=None
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().w4a16_gemm(_ptr(x), _ptr(packed_codes), _ptr(packed_scales), _ptr(y), M, N, K, _ptr(workspace),
                             ws_bytes, _stream(stream)), "w4a16_gemm")
+    return y
+
+
+def default_crossover_m() -> int:
+    """Largest M served by the W4A16 path when nvq_linear is given crossover < 0."""
+    return int(lib().nvq_default_crossover_m())
+
+
+def nvq_linear_workspace_bytes(M: int, N: int, K: int, crossover_m: int = -1) -> int:
+    return int(lib().nvq_linear_workspace_bytes(M, N, K, crossover_m))
+
+
+def nvq_linear(x, w4a4=None, w4a16=None, N: int | None = None, *, crossover_m: int = -1, y=None, workspace=None,
+               stream=None):
+    """Y [M, N] bf16 = X W^T through the path nvq_linear picks for this M.
+
+    w4a4: (codes, scales, t) of the NVFP4 master; w4a16: (packed_codes,
+    packed_scales) of the INT4 master; pass the form(s) the chosen path reads."""
+    _need_cuda(x)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+    M, K = x.shape
+    if N is None:
+        raise ValueError("N is required")
+    wc, wsc, wt = (None, None, None) if w4a4 is None else w4a4
+    pc, ps = (None, None) if w4a16 is None else w4a16
+    _need_cuda(wc, wsc, wt, pc, ps)
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    need = nvq_linear_workspace_bytes(M, N, K, crossover_m)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().nvq_linear(_ptr(x), M, N, K, _ptr(wc), _ptr(wsc), _ptr(wt), _ptr(pc), _ptr(ps), crossover_m,
+                            _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)), "nvq_linear")
     return y

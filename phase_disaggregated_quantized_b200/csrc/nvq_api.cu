@@ -124,6 +124,22 @@ nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* 
   return launch_status("w4a16_kernel");
 }
 
+// Workspace of nvq_linear's W4A4 path: activation codes, tiled scales, t and
+// the quantizer's scratch, each section 256-byte aligned.
+struct LinearWs {
+  size_t codes, scales, t, scratch, total;
+};
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+LinearWs linear_ws_layout(int64_t M, int64_t K) {
+  LinearWs L;
+  L.codes = 0;
+  L.scales = align256((size_t)M * (size_t)(K / 2));
+  L.t = L.scales + align256(nvfp4_scales_bytes(M, K));
+  L.scratch = L.t + 256;
+  L.total = L.scratch + align256(std::max<size_t>(16, nvfp4_quantize_workspace_bytes(M, K)));
+  return L;
+}
+
 }  // namespace
 
 extern "C" {
@@ -396,6 +412,45 @@ nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const voi
   if (M <= 8) return launch_w4a16<1>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
   if (M <= 16) return launch_w4a16<2>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
   return launch_w4a16<4>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
+}
+
+// ------------------------------------------------------------------ phase dispatch
+// Largest M at which W4A16 beat quantize + W4A4 on B200 for K = 4096, N = 24576
+// with weights read from HBM (profile_case --op crossover: 24.8 vs 30.2 us at
+// M = 8, 36.6 vs 29.2 us at M = 16).
+constexpr int64_t kDefaultCrossoverM = 8;
+
+int64_t nvq_default_crossover_m(void) { return kDefaultCrossoverM; }
+
+size_t nvq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t crossover_m) {
+  (void)N;
+  if (crossover_m < 0) crossover_m = kDefaultCrossoverM;
+  if (M <= crossover_m || M <= 0 || K <= 0 || K % 64 != 0) return 0;
+  return linear_ws_layout(M, K).total;
+}
+
+nvq_status nvq_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uint8_t* w_codes,
+                      const uint8_t* w_scales, const float* w_t, const uint8_t* w_packed_codes,
+                      const void* w_packed_scales, int64_t crossover_m, void* y_bf16, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (crossover_m < 0) crossover_m = kDefaultCrossoverM;
+  if (M <= crossover_m) {
+    if (!w_packed_codes || !w_packed_scales) return fail(NVQ_ERR_INVALID_ARG, "nvq_linear: W4A16 path needs the packed INT4 weights");
+    return w4a16_gemm(x_bf16, w_packed_codes, w_packed_scales, y_bf16, M, N, K, nullptr, 0, stream);
+  }
+  if (!w_codes || !w_scales || !w_t) return fail(NVQ_ERR_INVALID_ARG, "nvq_linear: W4A4 path needs the NVFP4 weights");
+  if (K <= 0 || K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvq_linear: W4A4 path needs K % 64 == 0");
+  if (N <= 0 || N % 8 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvq_linear: W4A4 path needs N % 8 == 0");
+  const LinearWs L = linear_ws_layout(M, K);
+  if (workspace == nullptr || workspace_bytes < L.total) return fail(NVQ_ERR_WORKSPACE, "nvq_linear: workspace too small");
+  if (!aligned16(workspace)) return fail(NVQ_ERR_MISALIGNED, "nvq_linear: workspace not 16-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* xc = ws + L.codes;
+  uint8_t* xs = ws + L.scales;
+  float* tx = reinterpret_cast<float*>(ws + L.t);
+  nvq_status st = nvfp4_quantize(x_bf16, M, K, nullptr, xc, xs, tx, ws + L.scratch, L.total - L.scratch, stream);
+  if (st != NVQ_OK) return st;
+  return nvfp4_gemm_w4a4(xc, xs, tx, w_codes, w_scales, w_t, y_bf16, M, N, K, stream);
 }
 
 }  // extern "C"

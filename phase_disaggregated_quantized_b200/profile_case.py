@@ -3,6 +3,7 @@
   python -m phase_disaggregated_quantized_b200.profile_case --op gemm --M 8192 --K 4096 --N 24576
   python -m phase_disaggregated_quantized_b200.profile_case --op w4a16 --M 1 --K 4096 --N 24576
   python -m phase_disaggregated_quantized_b200.profile_case --op quantize --M 8192 --K 12288
+  python -m phase_disaggregated_quantized_b200.profile_case --op crossover --K 4096 --N 24576
 
 Inputs are drawn on the GPU from the seeded generators; the offline steps
 (weight quantization and reorder) run once before the measured calls.  The
@@ -23,8 +24,8 @@ from phase_disaggregated_quantized_b200 import synth
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=("gemm", "w4a16", "quantize"), required=True)
-    ap.add_argument("--M", type=int, required=True)
+    ap.add_argument("--op", choices=("gemm", "w4a16", "quantize", "crossover"), required=True)
+    ap.add_argument("--M", type=int, default=0)
     ap.add_argument("--K", type=int, required=True)
     ap.add_argument("--N", type=int, default=0)
     ap.add_argument("--iters", type=int, default=3)
@@ -33,6 +34,8 @@ def main():
     a = ap.parse_args()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    if a.op == "crossover":
+        return crossover(a, dev)
     x = synth.activations_cuda(a.M, a.K, seed=11, device=dev)
     if a.op == "gemm":
         w = synth.weights_cuda(a.N, a.K, seed=11, device=dev)
@@ -85,6 +88,76 @@ def main():
     s = e0.elapsed_time(e1) / 1e3 / a.iters
     scale = 1e12 if unit == "TFLOP/s" else 1e9
     print(f"{a.op} M={a.M} K={a.K} N={a.N}: {1e6 * s:.2f} us/call, {work / s / scale:.1f} {unit}")
+
+
+def _graph_time(run, iters):
+    """Mean seconds per call of `iters` calls captured in one CUDA graph (after a warm replay)."""
+    run()
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(graph, stream=stream):
+            for _ in range(iters):
+                run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        graph.replay()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    nvq.check_device_error()
+    return e0.elapsed_time(e1) / 1e3 / iters
+
+
+def crossover(a, dev):
+    """Time both phase paths of one linear layer over a sweep of M (one BF16
+    master weight quantized both ways): W4A16 (weights INT4 g128, activations
+    BF16) against W4A4 (activations quantized to NVFP4 on the fly, then the
+    block-scaled GEMM).  Weights are cycled through enough copies to come from
+    HBM.  Prints one line per M and the largest M where W4A16 is faster."""
+    K, N = a.K, a.N or 24576
+    w = synth.weights_cuda(N, K, seed=5000, device=dev)
+    wq = nvq.nvfp4_quantize(w)
+    codes, scales = nvq.int4_quantize(w)
+    copies = max(1, -(-400_000_000 // (N * K // 2)))
+    packed = [nvq.int4_pack_weights(codes, scales, N, K) for _ in range(copies)]
+    fp4 = [wq] + [tuple(t.clone() for t in wq) for _ in range(copies - 1)]
+    del w
+    last_w4a16 = 0
+    rows = []
+    for M in (1, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 8192, 32768):
+        x = synth.activations_cuda(M, K, seed=5001, device=dev)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        xc = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+        xs = torch.empty(max(1, nvq.nvfp4_scales_bytes(M, K)), dtype=torch.uint8, device=dev)
+        tx = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.empty(max(16, nvq.nvfp4_quantize_workspace_bytes(M, K)), dtype=torch.uint8, device=dev)
+        k = [0]
+
+        def w4a16():
+            pc, ps = packed[k[0] % copies]
+            k[0] += 1
+            nvq.w4a16_gemm(x, pc, ps, N, y=y)
+
+        def w4a4():
+            wk = fp4[k[0] % copies]
+            k[0] += 1
+            nvq.nvfp4_quantize(x, None, codes=xc, scales=xs, tensor_scale_out=tx, workspace=ws)
+            nvq.nvfp4_gemm_w4a4((xc, xs, tx), wk, M, N, K, y=y)
+
+        iters = 8 if M <= 2048 else 3
+        t16 = _graph_time(w4a16, iters) if M <= 8192 else float("inf")
+        t4 = _graph_time(w4a4, iters)
+        if t16 < t4:
+            last_w4a16 = M
+        rows.append((M, t16, t4))
+        print(f"M={M:6d}  w4a16 {1e6 * t16:10.2f} us   w4a4+quantize {1e6 * t4:10.2f} us   "
+              f"faster: {'w4a16' if t16 < t4 else 'w4a4'}", flush=True)
+    print(f"crossover: W4A16 faster up to M = {last_w4a16} (K={K}, N={N})")
+    return rows
 
 
 if __name__ == "__main__":

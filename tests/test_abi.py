@@ -107,3 +107,29 @@ def test_product_path_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(root, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_phase_dispatch_host_rules(L):
+    """nvq_linear: path choice by M, workspace sizing and argument checks (no GPU)."""
+    c = L.nvq_default_crossover_m()
+    assert c >= 1
+    assert L.nvq_linear_workspace_bytes(c, 24576, 4096, -1) == 0               # W4A16 side: no scratch
+    big = L.nvq_linear_workspace_bytes(c + 1, 24576, 4096, -1)
+    assert big >= (c + 1) * 4096 // 2 + L.nvfp4_scales_bytes(c + 1, 4096)       # codes + scales at least
+    assert L.nvq_linear_workspace_bytes(64, 24576, 4096, 128) == 0              # caller's crossover wins
+    f = L.nvq_linear
+    # W4A16 side without the packed weights / W4A4 side without the NVFP4 weights
+    assert f(_vp(FAKE), 1, 256, 4096, _vp(FAKE), _vp(FAKE), _vp(FAKE), None, None, -1,
+             _vp(FAKE), None, 0, None) == 1
+    assert f(_vp(FAKE), 4096, 256, 4096, None, None, None, _vp(FAKE), _vp(FAKE), -1,
+             _vp(FAKE), _vp(FAKE), 1 << 30, None) == 1
+    # W4A4 side: workspace too small, misaligned, bad K
+    assert f(_vp(FAKE), 4096, 256, 4096, _vp(FAKE), _vp(FAKE), _vp(FAKE), None, None, -1,
+             _vp(FAKE), _vp(FAKE), 16, None) == 4
+    assert f(_vp(FAKE), 4096, 256, 4096, _vp(FAKE), _vp(FAKE), _vp(FAKE), None, None, -1,
+             _vp(FAKE), _vp(ODD), 1 << 30, None) == 3
+    assert f(_vp(FAKE), 4096, 256, 4100, _vp(FAKE), _vp(FAKE), _vp(FAKE), None, None, -1,
+             _vp(FAKE), _vp(FAKE), 1 << 30, None) == 2
+    # W4A16 side keeps its own shape rules (N % 16)
+    assert f(_vp(FAKE), 1, 24, 4096, None, None, None, _vp(FAKE), _vp(FAKE), -1,
+             _vp(FAKE), None, 0, None) == 2

@@ -338,5 +338,42 @@ def test_crossover_sweep_both_paths_sampled(M):
     assert ok, ("w4a16", M, worst)
 
 
+# ------------------------------------------------------------------ phase dispatch
+
+@pytest.mark.parametrize("M", [1, 8, 9, 40])
+def test_nvq_linear_dispatches_by_batch_size(M):
+    """One master W in both formats; nvq_linear must return exactly what the
+    path it picks returns, and that path must match its oracle."""
+    K, N = 512, 384
+    w = synth.weights(N, K, seed=77)
+    x = synth.activations(M, K, seed=78)
+    wq = gpu_quant(w)
+    packed = gpu_int4(w)
+    xg = x.cuda()
+    crossover = 8
+    y = nvq.nvq_linear(xg, wq, packed[2:], N, crossover_m=crossover)
+    nvq.check_device_error()
+    if M <= crossover:
+        direct = nvq.w4a16_gemm(xg, packed[2], packed[3], N)
+        got, ref = w4a16_case(x, w, packed)
+    else:
+        direct = nvq.nvfp4_gemm_w4a4(nvq.nvfp4_quantize(xg), wq, M, N, K)
+        got, ref = gemm_case(x, w)
+    nvq.check_device_error()
+    assert torch.equal(y, direct)
+    np.testing.assert_array_equal(bf16_to_f64(y), got)
+    ok, worst = onv.within_tolerance(got, ref)
+    assert ok, (M, worst)
+
+
+def test_nvq_linear_default_crossover_uses_w4a16_at_batch_one():
+    K, N = 4096, 4096
+    w = synth.weights(N, K, seed=79)
+    x = synth.activations(1, K, seed=80).cuda()
+    packed = gpu_int4(w)
+    y = nvq.nvq_linear(x, None, packed[2:], N)           # no NVFP4 form needed at M = 1
+    assert torch.equal(y, nvq.w4a16_gemm(x, packed[2], packed[3], N))
+
+
 def test_device_error_word_is_clear_after_normal_runs():
     nvq.check_device_error()
