@@ -232,6 +232,43 @@ nvq_status nvq_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K,
                       int64_t crossover_m, void* y_bf16, void* workspace, size_t workspace_bytes,
                       void* stream);
 
+/* ------------------------------------------------------------------------ *
+ * Prefill over layers whose NVFP4 weights live in pinned host memory
+ * (Disaggregated Quantization page, singularity-lens.com, its ODP scheme:
+ * prefill weights read layer block by layer block into two device buffers,
+ * the next read overlapping the current compute; here the weights come from
+ * pinned host memory, not from an SSD): layer l's
+ * weights are copied into device slot l % 2 on copy_stream while layer l - 1
+ * runs on compute_stream (activation quantize + W4A4 GEMM), so transfers and
+ * GEMMs overlap; a slot is refilled only after the GEMM that read it ended.
+ *
+ * Per layer: w_codes_host / w_scales_host / w_t_host as written by
+ * nvfp4_quantize for W [N, K] (N*K/2 bytes, nvfp4_scales_bytes(N, K) bytes,
+ * one float), in pinned host memory (cudaHostAlloc or registered); x_bf16 a
+ * device [M, K] BF16 input; y_bf16 a device [M, N] BF16 output.  Layers are
+ * independent (the caller chains them through x / y if it wants to).
+ * workspace: nvq_prefill_streamed_workspace_bytes(layers, n, M) device bytes,
+ * 16-byte aligned: two weight slots sized for the largest layer plus the
+ * activation quantizer's outputs and scratch.
+ * Both streams must belong to the current device; the call only enqueues work
+ * (it returns before the copies and kernels ran); the caller synchronises
+ * compute_stream before reading any y.  Shape rules: those of
+ * nvfp4_gemm_w4a4 per layer.  NULL pointers, bad shapes or a small
+ * workspace are reported before anything is enqueued.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const uint8_t* w_codes_host;
+  const uint8_t* w_scales_host;
+  const float* w_t_host;
+  const void* x_bf16;
+  void* y_bf16;
+  int64_t N, K;
+} nvq_stream_layer;
+
+size_t nvq_prefill_streamed_workspace_bytes(const nvq_stream_layer* layers, int n, int64_t M);
+nvq_status nvq_prefill_streamed(const nvq_stream_layer* layers, int n, int64_t M, void* workspace,
+                                size_t workspace_bytes, void* compute_stream, void* copy_stream);
+
 #ifdef __cplusplus
 }
 #endif

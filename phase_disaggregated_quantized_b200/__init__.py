@@ -31,6 +31,13 @@ STATUS = {0: "NVQ_OK", 1: "NVQ_ERR_INVALID_ARG", 2: "NVQ_ERR_UNSUPPORTED_SHAPE",
           4: "NVQ_ERR_WORKSPACE", 5: "NVQ_ERR_CUDA", 6: "NVQ_ERR_DEVICE_TIMEOUT"}
 
 
+class StreamLayer(ctypes.Structure):
+    """nvq_stream_layer of include/nvq.h."""
+    _fields_ = [("w_codes_host", ctypes.c_void_p), ("w_scales_host", ctypes.c_void_p),
+                ("w_t_host", ctypes.c_void_p), ("x_bf16", ctypes.c_void_p), ("y_bf16", ctypes.c_void_p),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
 class NvqError(RuntimeError):
     def __init__(self, status: int, where: str, detail: str = ""):
         self.status = status
@@ -70,6 +77,8 @@ def lib() -> ctypes.CDLL:
             "nvq_default_crossover_m": ([], i64),
             "nvq_linear_workspace_bytes": ([i64, i64, i64, i64], sz),
             "nvq_linear": ([vp, i64, i64, i64, vp, vp, vp, vp, vp, i64, vp, vp, sz, vp], i32),
+            "nvq_prefill_streamed_workspace_bytes": ([ctypes.POINTER(StreamLayer), i32, i64], sz),
+            "nvq_prefill_streamed": ([ctypes.POINTER(StreamLayer), i32, i64, vp, sz, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -234,3 +243,42 @@ def nvq_linear(x, w4a4=None, w4a16=None, N: int | None = None, *, crossover_m: i
     _check(lib().nvq_linear(_ptr(x), M, N, K, _ptr(wc), _ptr(wsc), _ptr(wt), _ptr(pc), _ptr(ps), crossover_m,
                             _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)), "nvq_linear")
     return y
+
+
+def _stream_layers(layers):
+    arr = (StreamLayer * len(layers))()
+    for i, L in enumerate(layers):
+        wc, ws, wt = L["w_host"]
+        for t in (wc, ws, wt):
+            if t.is_cuda or not t.is_pinned():
+                raise ValueError("streamed weights must be pinned host tensors")
+        _need_cuda(L["x"], L["y"])
+        arr[i] = StreamLayer(wc.data_ptr(), ws.data_ptr(), wt.data_ptr(), L["x"].data_ptr(), L["y"].data_ptr(),
+                             L["N"], L["K"])
+    return arr
+
+
+def prefill_streamed_workspace_bytes(layers, M: int) -> int:
+    return int(lib().nvq_prefill_streamed_workspace_bytes(_stream_layers(layers), len(layers), M))
+
+
+def prefill_streamed(layers, M: int, *, workspace=None, compute_stream=None, copy_stream=None):
+    """Run quantize + W4A4 GEMM for each layer with its NVFP4 weights copied from
+    pinned host memory into two device slots, copies overlapping the GEMMs.
+
+    layers: list of dicts with "w_host" (codes, scales, t as pinned CPU tensors
+    from nvfp4_quantize), "x" (device [M, K] bf16), "y" (device [M, N] bf16),
+    "N", "K".  Enqueues only; synchronise compute_stream before reading y."""
+    arr = _stream_layers(layers)
+    need = int(lib().nvq_prefill_streamed_workspace_bytes(arr, len(layers), M))
+    if workspace is None:
+        workspace = torch.empty(max(16, need), dtype=torch.uint8, device=layers[0]["x"].device)
+    if compute_stream is None:
+        compute_stream = torch.cuda.current_stream()
+    if copy_stream is None:
+        copy_stream = compute_stream
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().nvq_prefill_streamed(arr, len(layers), M, _ptr(workspace), ws_bytes,
+                                      ctypes.c_void_p(compute_stream.cuda_stream),
+                                      ctypes.c_void_p(copy_stream.cuda_stream)), "nvq_prefill_streamed")
+    return workspace

@@ -140,6 +140,44 @@ LinearWs linear_ws_layout(int64_t M, int64_t K) {
   return L;
 }
 
+// Workspace of nvq_prefill_streamed: two weight slots sized for the largest
+// layer (codes, tiled scales, t) and one set of activation quantizer outputs
+// sized for the largest K, sections 256-byte aligned.
+struct StreamWs {
+  bool ok = false;
+  size_t slot[2] = {0, 0};
+  size_t scales_off = 0, t_off = 0;                 // inside a slot
+  size_t act = 0;                                   // activation codes, then the rest
+  size_t act_scales_off = 0, act_t_off = 0, act_scratch_off = 0, act_scratch_bytes = 0;
+  size_t total = 0;
+};
+StreamWs stream_ws_layout(const nvq_stream_layer* layers, int n, int64_t M) {
+  StreamWs W;
+  size_t codes = 0, scales = 0, acodes = 0, ascales = 0, ascratch = 16;
+  for (int l = 0; l < n; ++l) {
+    const int64_t N = layers[l].N, K = layers[l].K;
+    if (N <= 0 || K <= 0 || N >= kMaxDim || K >= kMaxDim || M >= kMaxDim) return W;
+    codes = std::max(codes, (size_t)N * (size_t)(K / 2));
+    scales = std::max(scales, nvfp4_scales_bytes(N, K));
+    acodes = std::max(acodes, (size_t)M * (size_t)(K / 2));
+    ascales = std::max(ascales, nvfp4_scales_bytes(M, K));
+    ascratch = std::max(ascratch, nvfp4_quantize_workspace_bytes(M, K));
+  }
+  W.scales_off = align256(codes);
+  W.t_off = W.scales_off + align256(scales);
+  const size_t slot_bytes = W.t_off + 256;
+  W.slot[0] = 0;
+  W.slot[1] = slot_bytes;
+  W.act = 2 * slot_bytes;
+  W.act_scales_off = align256(acodes);
+  W.act_t_off = W.act_scales_off + align256(ascales);
+  W.act_scratch_off = W.act_t_off + 256;
+  W.act_scratch_bytes = align256(ascratch);
+  W.total = W.act + W.act_scratch_off + W.act_scratch_bytes;
+  W.ok = true;
+  return W;
+}
+
 }  // namespace
 
 extern "C" {
@@ -451,6 +489,77 @@ nvq_status nvq_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, const
   nvq_status st = nvfp4_quantize(x_bf16, M, K, nullptr, xc, xs, tx, ws + L.scratch, L.total - L.scratch, stream);
   if (st != NVQ_OK) return st;
   return nvfp4_gemm_w4a4(xc, xs, tx, w_codes, w_scales, w_t, y_bf16, M, N, K, stream);
+}
+
+// ------------------------------------------------------------------ prefill with host-resident weights
+size_t nvq_prefill_streamed_workspace_bytes(const nvq_stream_layer* layers, int n, int64_t M) {
+  if (layers == nullptr || n <= 0 || M < 0) return 0;
+  StreamWs W = stream_ws_layout(layers, n, M);
+  return W.ok ? W.total : 0;
+}
+
+nvq_status nvq_prefill_streamed(const nvq_stream_layer* layers, int n, int64_t M, void* workspace,
+                                size_t workspace_bytes, void* compute_stream_, void* copy_stream_) {
+  if (layers == nullptr || n <= 0 || M < 0) return fail(NVQ_ERR_INVALID_ARG, "nvq_prefill_streamed: bad layer list or M");
+  for (int l = 0; l < n; ++l) {
+    const nvq_stream_layer& L = layers[l];
+    if (!L.w_codes_host || !L.w_scales_host || !L.w_t_host || !L.x_bf16 || !L.y_bf16)
+      return fail(NVQ_ERR_INVALID_ARG, "nvq_prefill_streamed: NULL pointer in a layer");
+    if (L.N <= 0 || L.K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvq_prefill_streamed: bad layer sizes");
+    if (L.N % 8 != 0 || L.K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvq_prefill_streamed: need N % 8 == 0, K % 64 == 0");
+    if (M >= kMaxDim || L.N >= kMaxDim || L.K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvq_prefill_streamed: too large");
+    if (!aligned16(L.x_bf16) || !aligned16(L.y_bf16)) return fail(NVQ_ERR_MISALIGNED, "nvq_prefill_streamed: x / y not 16-byte aligned");
+  }
+  const StreamWs W = stream_ws_layout(layers, n, M);
+  if (!W.ok) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvq_prefill_streamed: sizes overflow");
+  if (workspace == nullptr || workspace_bytes < W.total) return fail(NVQ_ERR_WORKSPACE, "nvq_prefill_streamed: workspace too small");
+  if (!aligned16(workspace)) return fail(NVQ_ERR_MISALIGNED, "nvq_prefill_streamed: workspace not 16-byte aligned");
+  if (M == 0) return NVQ_OK;
+  cudaStream_t cs = static_cast<cudaStream_t>(compute_stream_), xs = static_cast<cudaStream_t>(copy_stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  // ready[s]: slot s holds the next layer's weights; freed[s]: the GEMM that read slot s ended.
+  cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
+  nvq_status st = NVQ_OK;
+  for (int s = 0; s < 2 && st == NVQ_OK; ++s) {
+    cudaError_t e = cudaEventCreateWithFlags(&ready[s], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&freed[s], cudaEventDisableTiming);
+    if (e != cudaSuccess) st = cuda_fail(e, "nvq_prefill_streamed: event");
+  }
+  if (st == NVQ_OK) {                            // work already queued on compute_stream may still read the slots
+    cudaError_t e = cudaEventRecord(freed[0], cs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(xs, freed[0], 0);
+    if (e != cudaSuccess) st = cuda_fail(e, "nvq_prefill_streamed: stream order");
+  }
+  for (int l = 0; l < n && st == NVQ_OK; ++l) {
+    const nvq_stream_layer& L = layers[l];
+    const int s = l & 1;
+    uint8_t* slot = ws + W.slot[s];
+    const size_t cb = (size_t)L.N * (size_t)(L.K / 2), sb = nvfp4_scales_bytes(L.N, L.K);
+    cudaError_t e = cudaSuccess;
+    if (l >= 2) e = cudaStreamWaitEvent(xs, freed[s], 0);       // the GEMM of layer l - 2 read this slot
+    if (e == cudaSuccess) e = cudaMemcpyAsync(slot, L.w_codes_host, cb, cudaMemcpyHostToDevice, xs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(slot + W.scales_off, L.w_scales_host, sb, cudaMemcpyHostToDevice, xs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(slot + W.t_off, L.w_t_host, sizeof(float), cudaMemcpyHostToDevice, xs);
+    if (e == cudaSuccess) e = cudaEventRecord(ready[s], xs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ready[s], 0);
+    if (e != cudaSuccess) { st = cuda_fail(e, "nvq_prefill_streamed: copy"); break; }
+    uint8_t* xc = ws + W.act;
+    uint8_t* xsc = xc + W.act_scales_off;
+    float* tx = reinterpret_cast<float*>(xc + W.act_t_off);
+    st = nvfp4_quantize(L.x_bf16, M, L.K, nullptr, xc, xsc, tx, xc + W.act_scratch_off, W.act_scratch_bytes, cs);
+    if (st == NVQ_OK)
+      st = nvfp4_gemm_w4a4(xc, xsc, tx, slot, slot + W.scales_off, reinterpret_cast<const float*>(slot + W.t_off),
+                           L.y_bf16, M, L.N, L.K, cs);
+    if (st == NVQ_OK) {
+      e = cudaEventRecord(freed[s], cs);
+      if (e != cudaSuccess) st = cuda_fail(e, "nvq_prefill_streamed: event record");
+    }
+  }
+  for (int s = 0; s < 2; ++s) {                  // released once the work recorded on them completes
+    if (ready[s]) cudaEventDestroy(ready[s]);
+    if (freed[s]) cudaEventDestroy(freed[s]);
+  }
+  return st;
 }
 
 }  // extern "C"

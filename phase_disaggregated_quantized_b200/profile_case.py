@@ -4,6 +4,7 @@
   python -m phase_disaggregated_quantized_b200.profile_case --op w4a16 --M 1 --K 4096 --N 24576
   python -m phase_disaggregated_quantized_b200.profile_case --op quantize --M 8192 --K 12288
   python -m phase_disaggregated_quantized_b200.profile_case --op crossover --K 4096 --N 24576
+  python -m phase_disaggregated_quantized_b200.profile_case --op streamed --M 8192 --layers 8
 
 Inputs are drawn on the GPU from the seeded generators; the offline steps
 (weight quantization and reorder) run once before the measured calls.  The
@@ -24,9 +25,10 @@ from phase_disaggregated_quantized_b200 import synth
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=("gemm", "w4a16", "quantize", "crossover"), required=True)
+    ap.add_argument("--op", choices=("gemm", "w4a16", "quantize", "crossover", "streamed"), required=True)
+    ap.add_argument("--layers", type=int, default=8, help="streamed: transformer layers of 4 Qwen3-8B linears")
     ap.add_argument("--M", type=int, default=0)
-    ap.add_argument("--K", type=int, required=True)
+    ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--N", type=int, default=0)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--copies", type=int, default=1,
@@ -36,6 +38,8 @@ def main():
     torch.cuda.set_device(dev)
     if a.op == "crossover":
         return crossover(a, dev)
+    if a.op == "streamed":
+        return streamed(a, dev)
     x = synth.activations_cuda(a.M, a.K, seed=11, device=dev)
     if a.op == "gemm":
         w = synth.weights_cuda(a.N, a.K, seed=11, device=dev)
@@ -158,6 +162,77 @@ def crossover(a, dev):
               f"faster: {'w4a16' if t16 < t4 else 'w4a4'}", flush=True)
     print(f"crossover: W4A16 faster up to M = {last_w4a16} (K={K}, N={N})")
     return rows
+
+
+def streamed(a, dev):
+    """Prefill over `layers` transformer layers (the four Qwen3-8B linears each)
+    with NVFP4 weights in pinned host memory: time the resident-weight pass,
+    the host->device copies alone, and nvq_prefill_streamed with the copies on
+    their own stream and on the compute stream."""
+    M = a.M or 8192
+    shapes = [(K, N) for _, K, N in synth.QWEN3_8B_LINEARS]
+    xs = {K: synth.activations_cuda(M, K, seed=6000 + K, device=dev) for K, _ in shapes}
+    ys = {(K, N): torch.empty(M, N, dtype=torch.bfloat16, device=dev) for K, N in shapes}
+    layers, resident, wbytes = [], [], 0
+    for li in range(a.layers):
+        for i, (K, N) in enumerate(shapes):
+            w = synth.weights_cuda(N, K, seed=7000 + 10 * li + i, device=dev)
+            wq = nvq.nvfp4_quantize(w)
+            del w
+            host = tuple(t.cpu().pin_memory() for t in wq)
+            wbytes += sum(t.numel() * t.element_size() for t in host)
+            layers.append(dict(w_host=host, x=xs[K], y=ys[(K, N)], N=N, K=K))
+            resident.append(wq)
+    torch.cuda.synchronize()
+    compute, copy = torch.cuda.current_stream(), torch.cuda.Stream()
+    ws = torch.empty(max(16, nvq.prefill_streamed_workspace_bytes(layers, M)), dtype=torch.uint8, device=dev)
+    dev_w = torch.empty(max(t.numel() * t.element_size() for L in layers for t in L["w_host"]), dtype=torch.uint8,
+                        device=dev)
+
+    def timed(fn, reps=3):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(compute)
+        for _ in range(reps):
+            fn()
+        copy_done = torch.cuda.Event()
+        copy_done.record(copy)
+        compute.wait_event(copy_done)
+        e1.record(compute)
+        torch.cuda.synchronize()
+        nvq.check_device_error()
+        return e0.elapsed_time(e1) / 1e3 / reps
+
+    def run_resident():
+        for L, wq in zip(layers, resident):
+            nvq.nvfp4_gemm_w4a4(nvq.nvfp4_quantize(L["x"]), wq, M, L["N"], L["K"], y=L["y"])
+
+    def run_copies():
+        copy.wait_stream(compute)
+        with torch.cuda.stream(copy):
+            for L in layers:
+                for t in L["w_host"]:
+                    dev_w[: t.numel() * t.element_size()].copy_(t.view(torch.uint8).view(-1), non_blocking=True)
+
+    def run_streamed():
+        nvq.prefill_streamed(layers, M, workspace=ws, compute_stream=compute, copy_stream=copy)
+
+    def run_serial():
+        nvq.prefill_streamed(layers, M, workspace=ws, compute_stream=compute, copy_stream=compute)
+
+    t_res = timed(run_resident)
+    t_copy = timed(run_copies)
+    t_str = timed(run_streamed)
+    t_ser = timed(run_serial)
+    flops = sum(2.0 * M * L["N"] * L["K"] for L in layers)
+    hidden = (t_res + t_copy - t_str) / min(t_res, t_copy)
+    print(f"M={M} layers={a.layers} linears={len(layers)} weights={wbytes / 1e6:.0f} MB (pinned host)")
+    print(f"resident weights : {1e3 * t_res:8.3f} ms  ({flops / t_res / 1e12:.0f} TFLOP/s)")
+    print(f"copies alone     : {1e3 * t_copy:8.3f} ms  ({wbytes / t_copy / 1e9:.1f} GB/s host->device)")
+    print(f"streamed, 2 strm : {1e3 * t_str:8.3f} ms  (bound max(resident, copies) = {1e3 * max(t_res, t_copy):.3f} ms)")
+    print(f"streamed, 1 strm : {1e3 * t_ser:8.3f} ms  (no overlap)")
+    print(f"overlap: {100 * hidden:.0f}% of the shorter of compute / copy hidden")
 
 
 if __name__ == "__main__":

@@ -133,3 +133,26 @@ def test_phase_dispatch_host_rules(L):
     # W4A16 side keeps its own shape rules (N % 16)
     assert f(_vp(FAKE), 1, 24, 4096, None, None, None, _vp(FAKE), _vp(FAKE), -1,
              _vp(FAKE), None, 0, None) == 2
+
+
+def test_prefill_streamed_host_rules(L):
+    """nvq_prefill_streamed: workspace sizing and argument checks (no GPU)."""
+    import phase_disaggregated_quantized_b200 as nvq
+    def layers(*shapes, bad=None):
+        arr = (nvq.StreamLayer * len(shapes))()
+        for i, (N, K) in enumerate(shapes):
+            arr[i] = nvq.StreamLayer(FAKE, FAKE, FAKE, FAKE, FAKE, N, K)
+        if bad is not None:
+            setattr(arr[0], bad, None)
+        return arr
+    one = L.nvq_prefill_streamed_workspace_bytes(layers((4096, 4096)), 1, 8192)
+    two = L.nvq_prefill_streamed_workspace_bytes(layers((4096, 4096), (24576, 4096)), 2, 8192)
+    assert one > 2 * 4096 * 2048 and two > one                      # two weight slots for the largest layer
+    assert two >= 2 * 24576 * 2048 + 8192 * 2048
+    s = L.nvq_prefill_streamed
+    assert s(layers((4096, 4096)), 0, 8192, _vp(FAKE), 1 << 40, None, None) == 1     # no layers
+    assert s(layers((4096, 4096), bad="w_t_host"), 1, 8192, _vp(FAKE), 1 << 40, None, None) == 1
+    assert s(layers((4100, 4096)), 1, 8192, _vp(FAKE), 1 << 40, None, None) == 2    # N % 8
+    assert s(layers((4096, 4100)), 1, 8192, _vp(FAKE), 1 << 40, None, None) == 2    # K % 64
+    assert s(layers((4096, 4096)), 1, 8192, _vp(FAKE), 16, None, None) == 4         # workspace
+    assert s(layers((4096, 4096)), 1, 8192, _vp(ODD), 1 << 40, None, None) == 3     # alignment

@@ -375,5 +375,37 @@ def test_nvq_linear_default_crossover_uses_w4a16_at_batch_one():
     assert torch.equal(y, nvq.w4a16_gemm(x, packed[2], packed[3], N))
 
 
+# ------------------------------------------------------------------ weights streamed from host
+
+def test_prefill_streamed_matches_resident_weights():
+    """Five layers with NVFP4 weights in pinned host memory, copies on their own
+    stream: every output equals the GEMM run on device-resident weights, also
+    when the same workspace is reused by a second call right away."""
+    M = 200
+    shapes = [(512, 256), (384, 512), (1024, 256), (256, 1024), (640, 384)]
+    layers, want = [], []
+    for i, (N, K) in enumerate(shapes):
+        w = synth.weights(N, K, seed=90 + i).cuda()
+        x = synth.activations(M, K, seed=95 + i).cuda()
+        wq = nvq.nvfp4_quantize(w)
+        want.append(nvq.nvfp4_gemm_w4a4(nvq.nvfp4_quantize(x), wq, M, N, K))
+        host = tuple(t.cpu().pin_memory() for t in wq)
+        layers.append(dict(w_host=host, x=x, y=torch.empty(M, N, dtype=torch.bfloat16, device="cuda"), N=N, K=K))
+    torch.cuda.synchronize()
+    copy_stream = torch.cuda.Stream()
+    ws = nvq.prefill_streamed(layers, M, copy_stream=copy_stream)
+    torch.cuda.synchronize()
+    nvq.check_device_error()
+    for L, ref in zip(layers, want):
+        assert torch.equal(L["y"], ref)
+    for L in layers:
+        L["y"].zero_()
+    nvq.prefill_streamed(layers, M, workspace=ws, copy_stream=copy_stream)
+    nvq.prefill_streamed(layers, M, workspace=ws, copy_stream=copy_stream)     # slots refilled while read?
+    torch.cuda.synchronize()
+    for L, ref in zip(layers, want):
+        assert torch.equal(L["y"], ref)
+
+
 def test_device_error_word_is_clear_after_normal_runs():
     nvq.check_device_error()
