@@ -13,6 +13,8 @@ Modules:
   int4      -- INT4 group-128 RTN quantization, W4A16 reference, the offline
                reorder and its inverse (MARLIN page).
   tiny_ref  -- independent pure-Python (Fraction) restatement for tiny inputs.
+  swiglu    -- gate_up GEMM + SiLU * mul + NVFP4 with a static tensor scale,
+               and the error-band comparison for its codes.
 
 Every function here is pinned by CPU tests against values fixed by the pages
 and by mathematics (closed forms, exhaustive brute force, hand-worked

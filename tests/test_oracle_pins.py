@@ -347,3 +347,69 @@ def test_marlin_scale_aware_bound_closed_form():
     r = int4.bytes_ratio_bf16_over_int4_g128()
     assert abs(r - 2.0 / (0.5 + 2.0 / 128)) < 1e-12
     assert 3.87 <= r < 3.88
+
+
+# ------------------------------------------------------------------ SiLU * mul epilogue (oracle/swiglu.py)
+
+def test_silu_closed_forms():
+    from oracle import swiglu
+    assert swiglu.silu(np.array([0.0]))[0] == 0.0
+    # silu(1) = 1 / (1 + e^-1), silu(-1) = -1 / (1 + e)
+    np.testing.assert_allclose(swiglu.silu(np.array([1.0, -1.0])),
+                               [1.0 / (1.0 + np.exp(-1.0)), -1.0 / (1.0 + np.e)], rtol=1e-15)
+    g = np.linspace(-30, 30, 601)
+    np.testing.assert_allclose(swiglu.silu(g) - swiglu.silu(-g), g, atol=1e-12)   # silu(g) - silu(-g) = g
+    assert swiglu.silu(np.array([800.0]))[0] == 800.0                              # sigmoid saturates at 1
+    assert swiglu.silu(np.array([-800.0]))[0] == 0.0
+
+
+def test_gate_up_reference_against_explicit_loops():
+    from oracle import swiglu
+    g = np.random.default_rng(5)
+    x = g.standard_normal((3, 32)); wg = g.standard_normal((4, 32)); wu = g.standard_normal((4, 32))
+    G, U, H = swiglu.gate_up_ref(x, wg, wu)
+    for m in range(3):
+        for n in range(4):
+            gv = sum(x[m, k] * wg[n, k] for k in range(32))
+            uv = sum(x[m, k] * wu[n, k] for k in range(32))
+            assert abs(G[m, n] - gv) < 1e-12 and abs(U[m, n] - uv) < 1e-12
+            assert abs(H[m, n] - gv / (1 + np.exp(-gv)) * uv) < 1e-12
+
+
+def test_consistency_check_accepts_exact_and_rejects_planted_errors():
+    from oracle import swiglu
+    rng = np.random.default_rng(6)
+    H = rng.standard_normal((4, 64)) * 3.0
+    t = float(np.float32(0.01))
+    codes, scales, _ = nvfp4.quantize(H, t_in=t)
+    zero = np.zeros_like(H)
+    ok, sr, cr = swiglu.consistent(codes, scales, H, zero, t)
+    assert ok and sr == 1.0 and cr == 1.0
+    bad = codes.copy()
+    i = np.argmax((bad & 7) <= 5)                              # a magnitude two steps away
+    bad.flat[i] = (bad.flat[i] & 8) | ((bad.flat[i] & 7) + 2)
+    assert not swiglu.consistent(bad, scales, H, np.full_like(H, 1e-9), t)[0]
+    flip = codes.copy()
+    j = np.argmax(np.abs(H) > 1.0)
+    flip.flat[j] ^= 8                                          # wrong sign on a clearly nonzero value
+    assert not swiglu.consistent(flip, scales, H, zero, t)[0]
+    s_bad = scales.copy()
+    s_bad[0, 0] += 3
+    assert not swiglu.consistent(codes, s_bad, H, zero, t)[0]
+
+
+def test_consistency_check_accepts_both_sides_of_a_threshold_inside_the_band():
+    from oracle import swiglu
+    t = 1.0
+    S = 8                                                      # E4M3 code 8 = 2^-6 ... pick the block scale
+    d = nvfp4.e4m3_value(S) * t
+    H = np.zeros((1, 16))
+    H[0, :] = 0.25 * d                                         # every element on midpoint 0 (tie -> code 0)
+    H[0, 0] = 6.0 * d                                          # block amax so the scale is exactly code S
+    codes, scales, _ = nvfp4.quantize(H, t_in=t)
+    assert scales[0, 0] == S and codes[0, 1] == 0
+    up = codes.copy()
+    up[0, 1] = 1                                               # the other side of the tie
+    band = np.full_like(H, 1e-3 * d)
+    assert swiglu.consistent(up, scales, H, band, t)[0]
+    assert not swiglu.consistent(up, scales, H, np.zeros_like(H), t)[0]
