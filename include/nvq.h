@@ -141,6 +141,33 @@ nvq_status nvfp4_gemm_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, cons
                            void* y_bf16, int64_t M, int64_t N, int64_t K, void* stream);
 
 /* ------------------------------------------------------------------------ *
+ * gate_up W4A4 GEMM whose epilogue applies SiLU * mul and writes NVFP4 for the
+ * down projection (Mix-Quant page, gist.science, section 2: NVFP4 activations
+ * with 16-element E4M3 scales and a tensor scale for the prefill linears; the
+ * Qwen3 gated MLP feeds down_proj with silu(x Wg^T) * (x Wu^T)).  The BF16
+ * [M, N] gate_up output never reaches memory.
+ *
+ *   G, U  = t_x t_w sum (NVFP4 products), FP32, as nvfp4_gemm_w4a4 computes Y
+ *   H     = silu(G) * U in FP32, silu(g) = g / (1 + exp(-g)) (relative error
+ *           about 1e-6 from the fast exponential and division)
+ *   codes, scales = NVFP4 RTN of H with the caller's static tensor scale *t_h
+ *           (the epilogue cannot see max|H| over the tensor before it writes),
+ *           the same exact rounding rules as nvfp4_quantize.
+ *
+ * w_codes / w_scales / t_w: nvfp4_quantize of the gate_up weight with its rows
+ * interleaved in blocks of 128: rows 256 b .. 256 b + 127 are gate rows
+ * 128 b .. 128 b + 127, the next 128 rows the same up rows (I = N / 2 gate and
+ * up rows each).  h_codes [M, I/2] bytes (even column in the low nibble);
+ * h_scales nvfp4_scales_bytes(M, I) bytes, tiled as nvfp4_quantize writes them
+ * (padding rows zero): the input nvfp4_gemm_w4a4 takes for down_proj, with
+ * t_x = *t_h.  Shape rules: N % 256 == 0, K % 64 == 0.
+ * ------------------------------------------------------------------------ */
+nvq_status nvfp4_gemm_w4a4_swiglu(const uint8_t* x_codes, const uint8_t* x_scales, const float* t_x,
+                                  const uint8_t* w_codes, const uint8_t* w_scales, const float* t_w,
+                                  const float* t_h, uint8_t* h_codes, uint8_t* h_scales, int64_t M, int64_t N,
+                                  int64_t K, void* stream);
+
+/* ------------------------------------------------------------------------ *
  * INT4 group-128 round-to-nearest weight quantization (MARLIN page: 4-bit
  * weights with one scale per 128-weight group).
  *

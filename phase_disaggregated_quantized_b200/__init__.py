@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
             "nvfp4_quantize": ([vp, i64, i64, vp, vp, vp, vp, vp, sz, vp], i32),
             "nvfp4_quantize_noalloc": ([vp, i64, i64, vp, vp, vp, vp, vp], i32),
             "nvfp4_gemm_w4a4": ([vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
+            "nvfp4_gemm_w4a4_swiglu": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
             "int4_quantize": ([vp, i64, i64, vp, vp, vp], i32),
             "int4_pack_weights": ([vp, vp, i64, i64, vp, vp, vp], i32),
             "w4a16_workspace_bytes": ([i64, i64, i64], sz),
@@ -168,6 +169,32 @@ def nvfp4_gemm_w4a4(xq, wq, M: int, N: int, K: int, *, y=None, stream=None):
     _check(lib().nvfp4_gemm_w4a4(_ptr(xc), _ptr(xs), _ptr(tx), _ptr(wc), _ptr(ws), _ptr(tw), _ptr(y), M, N, K,
                                  _stream(stream)), "nvfp4_gemm_w4a4")
     return y
+
+
+def interleave_gate_up(w_gate, w_up):
+    """[I, K] gate and up weights -> [2I, K] with rows interleaved in blocks of
+    128 (gate block b, then up block b), the order nvfp4_gemm_w4a4_swiglu reads."""
+    I, K = w_gate.shape
+    assert w_up.shape == (I, K) and I % 128 == 0
+    return torch.stack([w_gate.view(I // 128, 128, K), w_up.view(I // 128, 128, K)], dim=1).reshape(2 * I, K)
+
+
+def nvfp4_gemm_w4a4_swiglu(xq, wq, M: int, N: int, K: int, t_h, *, h_codes=None, h_scales=None, stream=None):
+    """NVFP4 H = silu(gate) * up of the gate_up GEMM (weight rows interleaved by
+    interleave_gate_up), quantized with the static tensor scale t_h (device
+    float tensor [1]).  Returns (h_codes [M, N/4] uint8, h_scales, t_h)."""
+    xc, xs, tx = xq
+    wc, ws, tw = wq
+    _need_cuda(xc, xs, tx, wc, ws, tw, t_h)
+    I = N // 2
+    if h_codes is None:
+        h_codes = torch.empty(M, I // 2, dtype=torch.uint8, device=xc.device)
+    if h_scales is None:
+        h_scales = torch.empty(max(1, nvfp4_scales_bytes(M, I)), dtype=torch.uint8, device=xc.device)
+    _check(lib().nvfp4_gemm_w4a4_swiglu(_ptr(xc), _ptr(xs), _ptr(tx), _ptr(wc), _ptr(ws), _ptr(tw), _ptr(t_h),
+                                        _ptr(h_codes), _ptr(h_scales), M, N, K, _stream(stream)),
+           "nvfp4_gemm_w4a4_swiglu")
+    return h_codes, h_scales, t_h
 
 
 def int4_quantize(w, *, codes=None, scales=None, stream=None):

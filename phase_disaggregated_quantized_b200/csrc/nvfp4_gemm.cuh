@@ -33,6 +33,7 @@
 // 32c + lane) and B scales at 16 + 8j .. 16 + 8j + 7 (column c: rows 32c + lane),
 // the same in all four sub-partitions.
 #pragma once
+#include "nvfp4_quantize.cuh"
 #include "ptx.cuh"
 
 namespace nvq {
@@ -82,6 +83,11 @@ struct Params {
   uint32_t k_atoms;        // K / 64: scale atoms per 128-row tile
   uint32_t n_row_atoms;    // padded N / 128
   uint32_t m_fastest;      // 1: tile index runs over row blocks first (A re-read per wave)
+  // SiLU * mul epilogue only (B rows interleaved in blocks of 128: gate, up, gate, up, ...)
+  uint8_t* h_codes;        // [M, N/2 / 2] E2M1 codes of H = silu(gate) * up
+  uint8_t* h_scales;       // tiled E4M3 scales of H, padded rows zero
+  const float* t_h;        // static tensor scale of H
+  uint32_t h_katoms;       // (N / 2) / 64
 };
 
 // Tile order: the tiles in flight at once (one per SM) cover a band of tiles
@@ -99,8 +105,100 @@ __device__ __forceinline__ void tile_coords(uint32_t tile, const Params& p, uint
   }
 }
 
+// ---------------------------------------------------------------- SiLU * mul -> NVFP4 epilogue
+// Per-CTA tables for the static tensor scale t_h of H, one entry per E4M3 block
+// scale code S: 1 / fl(S t_h), whether the fast map (fp32 product + cvt) gives
+// the exact RTN code for every fp32 input, and 6 x the midpoint to the next code.
+struct HTables {
+  float inv_d[128];
+  uint32_t fast_ok[128];
+  float mid6[128];
+};
+
+__device__ __forceinline__ uint32_t e2m1_code_f32(float x, float inv_d) {   // x >= 0
+  return e2m1x2_rn_satfinite(0.f, __fmul_rn(x, inv_d)) & 0xFu;
+}
+
+// Built by 127 threads.  The fast map is monotone in x, so it is exact for all
+// fp32 inputs once it is exact at the last fp32 below and the first fp32 at or
+// above every exact threshold mu_i S t (located with h = fl(P t) and the exact
+// residual fma(P, t, -h), P = mu_i S exact).
+__device__ __forceinline__ void build_h_table(HTables& tb, uint32_t c, float t) {
+  const float S = e4m3_value(c);
+  const float d = __fmul_rn(S, t);
+  const float inv = (c == 0) ? 0.f : __frcp_rn(d);
+  bool ok = (c == 0) || (d >= 1.17549435e-38f && !isinf(inv));
+  if (c != 0 && ok) {
+    for (int i = 0; i < 7 && ok; ++i) {
+      const float P = __fmul_rn(c_e2m1_mid[i], S);
+      const float h = __fmul_rn(P, t);
+      const float e = __fmaf_rn(P, t, -h);
+      if (isinf(h)) {
+        ok = e2m1_code_f32(3.40282347e38f, inv) == (uint32_t)i;
+        continue;
+      }
+      const bool pass_h = e < 0.f || (e == 0.f && ((i + 1) & 1) == 0);   // h above the threshold, or on a tie that goes up
+      const uint32_t hb = __float_as_uint(h);
+      const float x1 = pass_h ? h : __uint_as_float(hb + 1u);
+      if (e2m1_code_f32(x1, inv) != (uint32_t)(i + 1)) ok = false;
+      if (hb != 0u || !pass_h) {
+        const float x0 = pass_h ? __uint_as_float(hb - 1u) : h;
+        if (e2m1_code_f32(x0, inv) != (uint32_t)i) ok = false;
+      }
+    }
+  }
+  tb.inv_d[c] = inv;
+  tb.fast_ok[c] = ok ? 1u : 0u;
+  tb.mid6[c] = c < 126 ? __fmul_rn(6.0f, 0.5f * (S + e4m3_value(c + 1))) : 0.f;
+}
+
+// 16 fp32 values of one block -> 8 bytes of codes (even k in the low nibble)
+// and its E4M3 scale code.
+__device__ __forceinline__ uint32_t quantize_block16(const float (&v)[16], float t, float inv6t, const HTables& tb,
+                                                     uint2& out) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t s = block_scale_code(amax, t, inv6t, tb.mid6);
+  uint32_t w[2] = {0u, 0u};
+  if (tb.fast_ok[s]) {
+    const float inv = tb.inv_d[s];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {                          // signed product: the sign lands on the code
+      const uint32_t byte = e2m1x2_rn_satfinite(__fmul_rn(v[2 * i + 1], inv), __fmul_rn(v[2 * i], inv));
+      w[i >> 2] |= byte << (8 * (i & 3));
+    }
+  } else {
+    const float S = e4m3_value(s);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {                         // unrolled: v stays in registers
+      const float ax = fabsf(v[i]);
+      uint32_t mag = 0;
+      if (s != 0) {
+#pragma unroll
+        for (int j = 0; j < 7; ++j) {
+          const float r = __fmaf_rn(-__fmul_rn(c_e2m1_mid[j], S), t, ax);   // exact sign
+          mag += (r > 0.f || (r == 0.f && ((j + 1) & 1) == 0)) ? 1u : 0u;
+        }
+      }
+      const uint32_t code = mag | ((__float_as_uint(v[i]) >> 28) & 8u);
+      w[i >> 3] |= code << (4 * (i & 7));
+    }
+  }
+  out = make_uint2(w[0], w[1]);
+  return s;
+}
+
+// silu(g) * u in fp32.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
 __device__ __forceinline__ uint32_t acc_col(uint32_t buf) { return buf ? ACC1_COL : 0u; }
 
+// EPI 0: Y = BF16(alpha acc).  EPI 1: B rows interleaved in blocks of 128 (gate,
+// up, gate, up, ...); H = silu(gate) * up quantized to NVFP4 with a static t_h.
+template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                   const __grid_constant__ CUtensorMap tmap_y, const Params p) {
@@ -136,7 +234,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     fence_mbar_init();
     prefetch_tensormap(&tmap_a);
     prefetch_tensormap(&tmap_b);
-    prefetch_tensormap(&tmap_y);
+    if (EPI == 0) prefetch_tensormap(&tmap_y);
   }
   if (warp == 0) {
     tmem_alloc(smem_addr(tmem_ptr_smem), TMEM_COLS);
@@ -266,6 +364,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     const uint32_t h = (warp - 2) >> 2;                       // which 64-column chunk of each pair
     const uint32_t row = q * 32 + lane;                       // row of the tile held by this thread
     const float alpha = __ldg(p.t_x) * __ldg(p.t_w);
+    if constexpr (EPI == 0) {
     uint8_t* cbuf = smem + OFF_C + (warp - 2) * C_BYTES;      // this warp's 32 x 128 B staging
     const uint32_t cbuf_s = smem_addr(cbuf);
     uint32_t acc_par = 0, local = 0;
@@ -325,6 +424,72 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     if (lane == 0) bulk_wait<0>();
     __syncwarp();
     (void)row;
+    } else {
+      // SiLU * mul -> NVFP4.  Tile columns [0, 128) are gate rows of B, [128, 256)
+      // the matching up rows; this warp owns H columns 64 h .. 64 h + 63 of the
+      // tile (its gate chunk h and up chunk 2 + h) for rows 32 q .. 32 q + 31.
+      HTables& tb = *reinterpret_cast<HTables*>(smem + OFF_C);   // staging unused here
+      const float t_h = __ldg(p.t_h);
+      const uint32_t etid = threadIdx.x - 64u;                  // 0 .. 255 over the epilogue warps
+      if (etid < 127u) build_h_table(tb, etid, t_h);
+      named_barrier_sync(1, EPI_WARPS * 32);
+      const float inv6t = __frcp_rn(__fmul_rn(6.0f, t_h));
+      const uint32_t hrow_bytes = p.N >> 2;                     // (N / 2) codes, two per byte
+      uint32_t acc_par = 0, local = 0;
+      bool dead = false;
+      for (uint32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+        uint32_t mt, nt;
+        tile_coords(tile, p, mt, nt);
+        const uint32_t buf = local & 1u;
+        if (!dead && !warp_mbar_wait(bar_acc_full + 8 * buf, (acc_par >> buf) & 1u)) dead = true;
+        acc_par ^= 1u << buf;
+        if (dead) continue;
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + ((q * 32u) << 16) + acc_col(buf);
+        // The chunk in the region shared with the other accumulator first (up
+        // for accumulator 0, gate for accumulator 1), then the other in halves.
+        const uint32_t ch_first = (buf ? 0u : 2u) + h, ch_second = (buf ? 2u : 0u) + h;
+        uint32_t vf[64];
+        tc_ld_32x32b_x64(taddr + ch_first * C_COLS, vf);
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_overlap);
+        const uint32_t grow = mt * BM + row;
+        uint32_t sword = 0;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {              // unrolled: vf is indexed at compile time
+          uint32_t vs[32];
+          tc_ld_32x32b_x32(taddr + ch_second * C_COLS + 32u * part, vs);
+          tc_wait_ld();
+          if (part == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_acc_empty + 8 * buf);   // all of this tile's TMEM read
+          }
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            float hv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float a = __uint_as_float(vf[32 * part + 16 * b + i]) * alpha;
+              const float c2 = __uint_as_float(vs[16 * b + i]) * alpha;
+              hv[i] = buf ? silu_mul(a, c2) : silu_mul(c2, a);
+            }
+            uint2 codes;
+            const uint32_t sc = quantize_block16(hv, t_h, inv6t, tb, codes);
+            sword |= sc << (8 * (2 * part + b));
+            const uint32_t col = nt * 128u + h * 64u + 32u * part + 16u * b;   // H column of the block
+            if (grow < p.M) *reinterpret_cast<uint2*>(p.h_codes + (size_t)grow * hrow_bytes + (col >> 1)) = codes;
+          }
+        }
+        // The row's four scale bytes of blocks kb .. kb + 3: one aligned word of its atom.
+        const uint32_t kb = (nt * 128u + h * 64u) >> 4;
+        const size_t off = ((size_t)(grow >> 7) * p.h_katoms + (kb >> 2)) * 512u + (grow & 31u) * 16u +
+                           ((grow & 127u) >> 5) * 4u;
+        *reinterpret_cast<uint32_t*>(p.h_scales + off) = sword;
+      }
+    }
   }
 
   tc_fence_before();

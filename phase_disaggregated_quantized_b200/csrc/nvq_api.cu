@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "../../include/nvq.h"
@@ -327,17 +328,21 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const flo
 
 namespace {
 
+// EPI 0: y_bf16 receives Y.  EPI 1: h_* receive NVFP4(silu(gate) * up) with the
+// static scale t_h (B rows interleaved in blocks of 128: gate, up, ...).
+template <int EPI>
 nvq_status launch_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const float* t_x, const uint8_t* w_codes,
                        const uint8_t* w_scales, const float* t_w, void* y_bf16, int64_t M, int64_t N, int64_t K,
-                       cudaStream_t stream) {
+                       uint8_t* h_codes, uint8_t* h_scales, const float* t_h, cudaStream_t stream) {
   using namespace nvq::w4a4;
   CUtensorMap ma, mb, my;
+  memset(&my, 0, sizeof(my));                               // EPI 1 never touches Y
   if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
                    BKB, BM) ||
       !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
                    BKB, BN) ||
-      !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2,
-                   C_COLS, 32))                               // one epilogue warp: 32 rows x 64 columns
+      (EPI == 0 && !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, (uint64_t)N, (uint64_t)M,
+                                (uint64_t)N * 2, C_COLS, 32)))   // one epilogue warp: 32 rows x 64 columns
     return fail(NVQ_ERR_CUDA, "nvfp4_gemm_w4a4: tensor map encoding failed");
   Params p;
   p.x_scales = x_scales;
@@ -354,15 +359,19 @@ nvq_status launch_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const fl
   p.n_row_atoms = (uint32_t)((N + 127) / 128);
   // Sweep the smaller operand every wave (it stays in L2), stream the larger once.
   p.m_fastest = (uint64_t)M <= (uint64_t)N ? 1u : 0u;   // both operands have K/2 + K/16 bytes per row
+  p.h_codes = h_codes;
+  p.h_scales = h_scales;
+  p.t_h = t_h;
+  p.h_katoms = (uint32_t)(N / 2 / 64);
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    attr_err = cudaFuncSetAttribute(nvfp4_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "nvfp4_gemm_w4a4: smem attribute");
   const uint64_t tiles = (uint64_t)p.num_m_tiles * p.num_n_tiles;
   const int grid = (int)std::min<uint64_t>(tiles, (uint64_t)sm_count());
-  nvfp4_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, my, p);
+  nvfp4_gemm_kernel<EPI><<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, my, p);
   return launch_status("nvfp4_gemm_kernel");
 }
 
@@ -383,7 +392,28 @@ nvq_status nvfp4_gemm_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, cons
       !aligned16(y_bf16) || (reinterpret_cast<uintptr_t>(t_x) & 3u) || (reinterpret_cast<uintptr_t>(t_w) & 3u))
     return fail(NVQ_ERR_MISALIGNED, "nvfp4_gemm_w4a4: pointer not aligned");
   if (M == 0) return NVQ_OK;
-  return launch_w4a4(x_codes, x_scales, t_x, w_codes, w_scales, t_w, y_bf16, M, N, K, stream);
+  return launch_w4a4<0>(x_codes, x_scales, t_x, w_codes, w_scales, t_w, y_bf16, M, N, K, nullptr, nullptr, nullptr,
+                        stream);
+}
+
+nvq_status nvfp4_gemm_w4a4_swiglu(const uint8_t* x_codes, const uint8_t* x_scales, const float* t_x,
+                                  const uint8_t* w_codes, const uint8_t* w_scales, const float* t_w,
+                                  const float* t_h, uint8_t* h_codes, uint8_t* h_scales, int64_t M, int64_t N,
+                                  int64_t K, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4_swiglu: bad sizes");
+  if (N % 256 != 0 || K % 64 != 0)
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4_swiglu: need N % 256 == 0, K % 64 == 0");
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4_swiglu: too large");
+  if (!x_codes || !x_scales || !t_x || !w_codes || !w_scales || !t_w || !t_h || !h_codes || !h_scales)
+    return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4_swiglu: NULL pointer");
+  if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(h_codes) || !aligned16(h_scales) || (reinterpret_cast<uintptr_t>(t_x) & 3u) ||
+      (reinterpret_cast<uintptr_t>(t_w) & 3u) || (reinterpret_cast<uintptr_t>(t_h) & 3u))
+    return fail(NVQ_ERR_MISALIGNED, "nvfp4_gemm_w4a4_swiglu: pointer not aligned");
+  if (M == 0) return NVQ_OK;
+  return launch_w4a4<1>(x_codes, x_scales, t_x, w_codes, w_scales, t_w, nullptr, M, N, K, h_codes, h_scales, t_h,
+                        stream);
 }
 
 // ------------------------------------------------------------------ INT4

@@ -5,6 +5,7 @@
   python -m phase_disaggregated_quantized_b200.profile_case --op quantize --M 8192 --K 12288
   python -m phase_disaggregated_quantized_b200.profile_case --op crossover --K 4096 --N 24576
   python -m phase_disaggregated_quantized_b200.profile_case --op streamed --M 8192 --layers 8
+  python -m phase_disaggregated_quantized_b200.profile_case --op swiglu --M 8192 --K 4096 --N 24576
 
 Inputs are drawn on the GPU from the seeded generators; the offline steps
 (weight quantization and reorder) run once before the measured calls.  The
@@ -25,7 +26,7 @@ from phase_disaggregated_quantized_b200 import synth
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=("gemm", "w4a16", "quantize", "crossover", "streamed"), required=True)
+    ap.add_argument("--op", choices=("gemm", "w4a16", "quantize", "crossover", "streamed", "swiglu"), required=True)
     ap.add_argument("--layers", type=int, default=8, help="streamed: transformer layers of 4 Qwen3-8B linears")
     ap.add_argument("--M", type=int, default=0)
     ap.add_argument("--K", type=int, default=4096)
@@ -40,6 +41,8 @@ def main():
         return crossover(a, dev)
     if a.op == "streamed":
         return streamed(a, dev)
+    if a.op == "swiglu":
+        return swiglu(a, dev)
     x = synth.activations_cuda(a.M, a.K, seed=11, device=dev)
     if a.op == "gemm":
         w = synth.weights_cuda(a.N, a.K, seed=11, device=dev)
@@ -233,6 +236,45 @@ def streamed(a, dev):
     print(f"streamed, 2 strm : {1e3 * t_str:8.3f} ms  (bound max(resident, copies) = {1e3 * max(t_res, t_copy):.3f} ms)")
     print(f"streamed, 1 strm : {1e3 * t_ser:8.3f} ms  (no overlap)")
     print(f"overlap: {100 * hidden:.0f}% of the shorter of compute / copy hidden")
+
+
+def swiglu(a, dev):
+    """gate_up GEMM with the SiLU * mul -> NVFP4 epilogue against the same GEMM
+    writing BF16 and against the unfused chain (BF16 GEMM, then silu * mul by
+    torch, then nvfp4_quantize of H with the same static scale)."""
+    M, K, N = a.M or 8192, a.K, a.N or 24576
+    I = N // 2
+    x = synth.activations_cuda(M, K, seed=8000, device=dev)
+    wg = synth.weights_cuda(I, K, seed=8001, device=dev)
+    wu = synth.weights_cuda(I, K, seed=8002, device=dev)
+    wi = nvq.interleave_gate_up(wg, wu).contiguous()
+    wc = torch.cat([wg, wu])                                   # gate rows, then up rows (plain layout)
+    del wg, wu
+    xq, wqi, wqc = nvq.nvfp4_quantize(x), nvq.nvfp4_quantize(wi), nvq.nvfp4_quantize(wc)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    t_h = torch.tensor([0.02], dtype=torch.float32, device=dev)
+    hc = torch.empty(M, I // 2, dtype=torch.uint8, device=dev)
+    hs = torch.empty(nvq.nvfp4_scales_bytes(M, I), dtype=torch.uint8, device=dev)
+    ht = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def fused():
+        nvq.nvfp4_gemm_w4a4_swiglu(xq, wqi, M, N, K, t_h, h_codes=hc, h_scales=hs)
+
+    def plain():
+        nvq.nvfp4_gemm_w4a4(xq, wqc, M, N, K, y=y)
+
+    def unfused():
+        nvq.nvfp4_gemm_w4a4(xq, wqc, M, N, K, y=y)
+        h = torch.nn.functional.silu(y[:, :I]) * y[:, I:]
+        nvq.nvfp4_quantize(h, t_h, codes=hc, scales=hs, tensor_scale_out=ht)
+
+    flops = 2.0 * M * N * K
+    tf, tp, tu = _graph_time(fused, 5), _graph_time(plain, 5), _graph_time(unfused, 5)
+    print(f"M={M} K={K} N={N} (I={I})")
+    print(f"fused SiLU*mul -> NVFP4 epilogue : {1e6 * tf:9.1f} us  {flops / tf / 1e12:7.0f} TFLOP/s")
+    print(f"same GEMM, BF16 output           : {1e6 * tp:9.1f} us  {flops / tp / 1e12:7.0f} TFLOP/s")
+    print(f"unfused: BF16 GEMM + silu*mul + quantize : {1e6 * tu:9.1f} us")
+    print(f"H bytes written: fused {M * I // 2 + M * I // 16} vs BF16 Y {2 * M * N}")
 
 
 if __name__ == "__main__":

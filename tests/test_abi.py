@@ -156,3 +156,17 @@ def test_prefill_streamed_host_rules(L):
     assert s(layers((4096, 4100)), 1, 8192, _vp(FAKE), 1 << 40, None, None) == 2    # K % 64
     assert s(layers((4096, 4096)), 1, 8192, _vp(FAKE), 16, None, None) == 4         # workspace
     assert s(layers((4096, 4096)), 1, 8192, _vp(ODD), 1 << 40, None, None) == 3     # alignment
+
+
+def test_swiglu_gemm_host_rules(L):
+    f = L.nvfp4_gemm_w4a4_swiglu
+    P = [_vp(FAKE)] * 9
+    assert f(*P, 128, 384, 512, None) == 2                   # N % 256
+    assert f(*P, 128, 512, 100, None) == 2                   # K % 64
+    Pn = list(P)
+    Pn[6] = None                                             # t_h
+    assert f(*Pn, 128, 512, 512, None) == 1
+    Pm = list(P)
+    Pm[7] = _vp(ODD)                                         # h_codes misaligned
+    assert f(*Pm, 128, 512, 512, None) == 3
+    assert f(*P, 0, 512, 512, None) == 0                     # M = 0: nothing to do

@@ -375,6 +375,66 @@ def test_nvq_linear_default_crossover_uses_w4a16_at_batch_one():
     assert torch.equal(y, nvq.w4a16_gemm(x, packed[2], packed[3], N))
 
 
+# ------------------------------------------------------------------ gate_up GEMM with SiLU * mul -> NVFP4
+
+def _swiglu_case(M, I, K, seed, rows=None, t_scale=1.0, gpu_inputs=False):
+    """Runs the fused kernel and returns what the oracle comparison needs."""
+    from oracle import swiglu as osw
+    gen = synth.activations_cuda if gpu_inputs else synth.activations
+    wgen = synth.weights_cuda if gpu_inputs else synth.weights
+    x = gen(M, K, seed=seed)
+    wg, wu = wgen(I, K, seed=seed + 1), wgen(I, K, seed=seed + 2)
+    wi = nvq.interleave_gate_up(wg.cuda(), wu.cuda()).contiguous()
+    xq = gpu_quant(x)
+    wq = gpu_quant(wi)
+    x_cpu = x.cpu()
+    wg_c, wu_c = wg.cpu(), wu.cpu()
+    tx = onv.tensor_scale_from_amax(float(x_cpu.abs().max()))
+    tw = onv.tensor_scale_from_amax(float(torch.maximum(wg_c.abs().max(), wu_c.abs().max())))
+    assert float(xq[2].item()) == tx and float(wq[2].item()) == tw
+    rows = np.arange(M) if rows is None else rows
+    xc, xs, _ = onv.quantize(bf16_to_f64(x_cpu[torch.tensor(rows)]), t_in=tx)
+    gc, gs, _ = onv.quantize(bf16_to_f64(wg_c), t_in=tw)
+    uc, us, _ = onv.quantize(bf16_to_f64(wu_c), t_in=tw)
+    xh = onv.dequantize(xc, xs, tx)
+    G, U, H = osw.gate_up_ref(xh, onv.dequantize(gc, gs, tw), onv.dequantize(uc, us, tw))
+    t_h = float(np.float32(t_scale * float(np.max(np.abs(H))) / 2688.0))
+    th_dev = torch.tensor([t_h], dtype=torch.float32, device="cuda")
+    hc, hs, _ = nvq.nvfp4_gemm_w4a4_swiglu(xq, wq, M, 2 * I, K, th_dev)
+    nvq.check_device_error()
+    codes = onv.unpack_codes(u8(hc))[rows]
+    scales = onv.scales_from_tiled(u8(hs), M, I)[rows]
+    return osw.consistent(codes, scales, H, osw.error_band(G, U), t_h), u8(hs), M, I
+
+
+@pytest.mark.parametrize("M,I,K,t_scale", [(200, 256, 256, 1.0), (128, 384, 512, 1.0), (72, 128, 64, 1.0),
+                                           (130, 256, 320, 0.05), (64, 256, 256, 40.0)])
+def test_swiglu_gemm_emits_valid_nvfp4(M, I, K, t_scale):
+    """Every block scale and code is the exact RTN result for some H' inside the
+    GEMM error band of the oracle's H; nearly all agree with the oracle's own
+    RTN of H.  t_scale < 1 saturates many blocks at the largest scale, > 1
+    sends small blocks to zero scales."""
+    (ok, s_rate, c_rate), hs, M_, I_ = _swiglu_case(M, I, K, seed=300 + M + K, t_scale=t_scale)
+    assert ok
+    assert s_rate >= 0.99 and c_rate >= 0.99, (s_rate, c_rate)
+    full = onv.scales_from_tiled(hs, M_, I_)
+    assert full.shape == (M_, I_ // 16)
+    pad = onv.padded_rows(M_)
+    if pad > M_:                                             # padding rows of the tiled layout are zero
+        offs = onv.scale_offsets(pad, I_)[M_:]
+        assert not hs[offs].any()
+
+
+def test_swiglu_gemm_qwen3_8b_gate_up_full_size_sampled():
+    """M = 8192, K = 4096, I = 12288 (gate_up N = 24576): 24 sampled rows, every
+    H column of those rows."""
+    g = np.random.default_rng(9)
+    rows = np.sort(g.choice(8192, 24, replace=False))
+    (ok, s_rate, c_rate), _, _, _ = _swiglu_case(8192, 12288, 4096, seed=5100, rows=rows, gpu_inputs=True)
+    assert ok
+    assert s_rate >= 0.99 and c_rate >= 0.99, (s_rate, c_rate)
+
+
 # ------------------------------------------------------------------ weights streamed from host
 
 def test_prefill_streamed_matches_resident_weights():
