@@ -15,6 +15,8 @@ Modules:
   tiny_ref  -- independent pure-Python (Fraction) restatement for tiny inputs.
   swiglu    -- gate_up GEMM + SiLU * mul + NVFP4 with a static tensor scale,
                and the error-band comparison for its codes.
+  sparse24  -- 2:4 magnitude pruning + INT4 group-128, the sparse W4A16
+               reference, and the decode kernel's packed order with its inverse.
 
 Every function here is pinned by CPU tests against values fixed by the pages
 and by mathematics (closed forms, exhaustive brute force, hand-worked

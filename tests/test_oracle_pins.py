@@ -413,3 +413,86 @@ def test_consistency_check_accepts_both_sides_of_a_threshold_inside_the_band():
     band = np.full_like(H, 1e-3 * d)
     assert swiglu.consistent(up, scales, H, band, t)[0]
     assert not swiglu.consistent(up, scales, H, np.zeros_like(H), t)[0]
+
+
+# ------------------------------------------------------------------ 2:4 sparse INT4 (oracle/sparse24.py)
+
+def test_prune24_keeps_two_largest_per_run_with_lower_index_on_ties():
+    from oracle import sparse24
+    w = np.array([[1.0, -3.0, 2.0, 0.5, 0.0, 0.0, 0.0, 0.0, 2.0, -2.0, 2.0, 1.0, -1.0, 1.0, 1.0, -1.0]])
+    pruned, keep = sparse24.prune24(w)
+    np.testing.assert_array_equal(keep[0], [0, 1, 1, 0, 1, 1, 0, 0, 1, 1, 0, 0, 1, 1, 0, 0])
+    np.testing.assert_array_equal(pruned[0], [0, -3, 2, 0, 0, 0, 0, 0, 2, -2, 0, 0, -1, 1, 0, 0])
+    g = np.random.default_rng(7)
+    w = np.round(g.standard_normal((6, 64)) * 4) / 4                # many exact ties
+    pruned, keep = sparse24.prune24(w)
+    kr, ar = keep.reshape(6, 16, 4), np.abs(w).reshape(6, 16, 4)
+    assert np.all(kr.sum(axis=2) == 2)
+    for n in range(6):                                            # brute force over the 6 choices
+        for r in range(16):
+            best = max(((ar[n, r, a] + ar[n, r, b], -a, -b), (a, b)) for a in range(4) for b in range(a + 1, 4))
+            a, b = best[1]
+            assert kr[n, r, a] and kr[n, r, b]
+
+
+def test_sparse_quantize_matches_dense_int4_of_the_pruned_weight():
+    from oracle import sparse24
+    w = synth_like(32, 256, seed=8)
+    u_kept, meta, s_bits, keep = sparse24.quantize(w)
+    pruned, _ = sparse24.prune24(w)
+    u_dense, s_dense = int4.quantize(pruned)
+    np.testing.assert_array_equal(sparse24.dense_codes(u_kept, meta), u_dense)
+    np.testing.assert_array_equal(s_bits, s_dense)
+    _, s_unpruned = int4.quantize(w)                              # a run's max is kept: same scales
+    np.testing.assert_array_equal(s_bits, s_unpruned)
+    i0, i1 = meta & 3, meta >> 2
+    assert np.all(i0 < i1)
+
+
+def test_sparse_pack_is_a_bijection_and_matches_hand_slots():
+    from oracle import sparse24
+    g = np.random.default_rng(9)
+    N, K = 32, 256
+    u = g.integers(0, 16, size=(N, K // 2)).astype(np.uint8)
+    pairs = np.array([a | (b << 2) for a in range(4) for b in range(a + 1, 4)], dtype=np.uint8)
+    meta = pairs[g.integers(0, 6, size=(N, K // 4))]
+    s = g.integers(0, 1 << 16, size=(N, K // 128)).astype(np.uint16)
+    p, ps = sparse24.pack(u, meta, s)
+    assert p.size == (N // 16) * (K // 128) * 768 and ps.size == (N // 16) * (K // 128) * 32
+    u2, m2, s2 = sparse24.unpack(p, ps, N, K)
+    np.testing.assert_array_equal(u2, u)
+    np.testing.assert_array_equal(m2, meta)
+    np.testing.assert_array_equal(s2, s)
+    words = p[:512].copy().view(np.uint32)
+    kr = u.reshape(N, K // 4, 2)
+    w0 = int(words[0])                                            # lane 0, step 0
+    assert (w0 & 0xF) == kr[0, 0, 0] and ((w0 >> 16) & 0xF) == kr[0, 0, 1]     # row 0, run 0
+    assert ((w0 >> 4) & 0xF) == kr[8, 0, 0]                                     # row 8, run 0
+    assert ((w0 >> 8) & 0xF) == kr[0, 2, 0] and ((w0 >> 24) & 0xF) == kr[0, 2, 1]   # compressed k 8, 9: run 2
+    w = int(words[4 * 5 + 3])                                     # lane 5 (g 1, c 1), step 3
+    assert (w & 0xF) == kr[1, 8 * 3 + 4, 0]                       # compressed k 2: MMA run 1 -> run 8*3+4
+    m = p[512:].copy().view(np.uint32)
+    m0 = int(m[0])                                                # lane (0, 0), step 0
+    assert (m0 & 0xF) == meta[0, 0] and ((m0 >> 4) & 0xF) == meta[0, 4] and ((m0 >> 16) & 0xF) == meta[8, 0]
+    m1 = int(m[4 * 1 + 2])                                        # lane (0, 1), step 2: MMA runs 4..7
+    assert (m1 & 0xF) == meta[0, 16 + 2] and ((m1 >> 4) & 0xF) == meta[0, 16 + 6]
+
+
+def test_sparse_w4a16_reference_against_explicit_loops():
+    from oracle import sparse24
+    w = synth_like(16, 128, seed=10)
+    x = np.random.default_rng(11).standard_normal((2, 128))
+    u_kept, meta, s_bits, keep = sparse24.quantize(w)
+    y = sparse24.w4a16_ref(x, u_kept, meta, s_bits)
+    s = int4.bf16_bits_to_f64(s_bits)
+    u = sparse24.dense_codes(u_kept, meta).astype(np.int64)
+    for m in range(2):
+        for n in range(16):
+            ref = sum(x[m, k] * s[n, 0] * (u[n, k] - 8) for k in range(128) if keep[n, k])
+            assert abs(y[m, n] - ref) < 1e-9
+
+
+def synth_like(N, K, seed):
+    """bf16-valued float64 weights 0.02 N(0,1) (the pins need only values on the bf16 grid)."""
+    v = np.random.default_rng(seed).standard_normal((N, K)) * 0.02
+    return int4.bf16_bits_to_f64(int4.f64_to_bf16_bits_rne(v))
