@@ -229,6 +229,29 @@ nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const voi
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------ *
+ * 2:4-sparse INT4 decode (MARLIN page, abeam.tech: its official implementation
+ * also combines the group-128 INT4 weights with 2:4 structured sparsity).
+ *
+ * int4_pack_sparse24 prunes the BF16 master W [N, K] 2:4 (in every run of 4
+ * consecutive k of a row the 2 entries of largest |w| stay, the lower k winning
+ * among equal magnitudes) and writes the kept INT4 codes in the order of the
+ * m16n8k32 sparse MMA, with their 2-bit positions as MMA metadata.  codes and
+ * scales_bf16 are int4_quantize of the same W (a run's largest |w| is always
+ * kept, so the group scales and the kept codes equal the dense ones).
+ * packed: N*K*3/8 bytes (per 16-row x 128-k unit: 512 bytes of codes, 256 of
+ * metadata); packed_scales: N*(K/128)*2 bytes, the layout of int4_pack_weights.
+ *
+ * w4a16_sparse24_gemm: Y = X (s (u - 8) at the kept positions, 0 elsewhere)^T,
+ * with the arithmetic of w4a16_gemm (exact products, FP32 sums, group scale in
+ * FP32, BF16 RNE out) and its streaming kernel on 24% fewer weight bytes.
+ * Shape rules for both: N % 16 == 0, K % 128 == 0; pointers 16-byte aligned.
+ * ------------------------------------------------------------------------ */
+nvq_status int4_pack_sparse24(const void* w_bf16, const uint8_t* codes, const void* scales_bf16, int64_t N,
+                              int64_t K, uint8_t* packed, void* packed_scales, void* stream);
+nvq_status w4a16_sparse24_gemm(const void* x_bf16, const uint8_t* packed, const void* packed_scales,
+                               void* y_bf16, int64_t M, int64_t N, int64_t K, void* stream);
+
+/* ------------------------------------------------------------------------ *
  * Phase dispatch over one master weight held in both formats (Disaggregated
  * Quantization page, singularity-lens.com, the section on format
  * disaggregation; Mix-Quant page, gist.science, section 2: NVFP4 W4A4 where

@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
             "int4_pack_weights": ([vp, vp, i64, i64, vp, vp, vp], i32),
             "w4a16_workspace_bytes": ([i64, i64, i64], sz),
             "w4a16_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp, sz, vp], i32),
+            "int4_pack_sparse24": ([vp, vp, vp, i64, i64, vp, vp, vp], i32),
+            "w4a16_sparse24_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp], i32),
             "nvq_default_crossover_m": ([], i64),
             "nvq_linear_workspace_bytes": ([i64, i64, i64, i64], sz),
             "nvq_linear": ([vp, i64, i64, i64, vp, vp, vp, vp, vp, i64, vp, vp, sz, vp], i32),
@@ -235,6 +237,32 @@ def w4a16_gemm(x, packed_codes, packed_scales, N: int, *, y=None, workspace=None
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().w4a16_gemm(_ptr(x), _ptr(packed_codes), _ptr(packed_scales), _ptr(y), M, N, K, _ptr(workspace),
                             ws_bytes, _stream(stream)), "w4a16_gemm")
+    return y
+
+
+def int4_pack_sparse24(w, codes, scales, *, packed=None, packed_scales=None, stream=None):
+    """2:4-prune the BF16 master w [N, K] and pack its kept INT4 codes (from
+    int4_quantize(w)) for w4a16_sparse24_gemm."""
+    _need_cuda(w, codes, scales)
+    N, K = w.shape
+    if packed is None:
+        packed = torch.empty(N * K * 3 // 8, dtype=torch.uint8, device=w.device)
+    if packed_scales is None:
+        packed_scales = torch.empty(N * (K // 128) * 2, dtype=torch.uint8, device=w.device)
+    _check(lib().int4_pack_sparse24(_ptr(w), _ptr(codes), _ptr(scales), N, K, _ptr(packed), _ptr(packed_scales),
+                                    _stream(stream)), "int4_pack_sparse24")
+    return packed, packed_scales
+
+
+def w4a16_sparse24_gemm(x, packed, packed_scales, N: int, *, y=None, stream=None):
+    """BF16 X [M, K] times the 2:4-sparse packed INT4 W [N, K] -> Y [M, N] bf16."""
+    _need_cuda(x, packed, packed_scales)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+    M, K = x.shape
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _check(lib().w4a16_sparse24_gemm(_ptr(x), _ptr(packed), _ptr(packed_scales), _ptr(y), M, N, K, _stream(stream)),
+           "w4a16_sparse24_gemm")
     return y
 
 

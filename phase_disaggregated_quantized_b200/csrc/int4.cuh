@@ -93,3 +93,85 @@ __global__ void int4_pack_kernel(const uint8_t* __restrict__ codes, const uint16
 }
 
 }  // namespace nvq
+
+namespace nvq {
+
+// ---------------------------------------------------------------- 2:4 sparse packing
+// 2:4 magnitude pruning of the BF16 master (two largest |w| of every run of four
+// k, the lower k on equal magnitudes) combined with the dense INT4 codes (a
+// run's largest |w| is always kept, so the group scales and the kept codes are
+// the dense ones), written in the sparse decode kernel's order: per 16-row x
+// 128-k unit, 512 bytes of A-fragment code words (lane-major, 4 m16n8k32 steps
+// per lane) and 256 bytes of metadata words (lanes c = 0, 1), then the unit's
+// 32 bytes of scales as in int4_pack_kernel.
+
+// Kept positions (i0 < i1) of one run from its four bf16 values.
+__device__ __forceinline__ uint32_t run_meta(uint2 w4) {
+  const uint32_t a[4] = {w4.x & 0x7FFFu, (w4.x >> 16) & 0x7FFFu, w4.y & 0x7FFFu, (w4.y >> 16) & 0x7FFFu};
+  uint32_t keep = 0;
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    uint32_t beaten = 0;                                   // runs ahead of p in the (|w| desc, k asc) order
+#pragma unroll
+    for (int q = 0; q < 4; ++q) beaten += (a[q] > a[p] || (a[q] == a[p] && q < p)) ? 1u : 0u;
+    if (beaten < 2) keep |= 1u << p;
+  }
+  const uint32_t i0 = __ffs(keep) - 1, i1 = 31 - __clz(keep);
+  return i0 | (i1 << 2);
+}
+
+// MMA step s, MMA run j -> run of the 128-k group.
+__device__ __forceinline__ uint32_t sparse_run(uint32_t s, uint32_t j) {
+  return 8 * s + ((j & 1u) ? 4 + (j >> 1) : (j >> 1));
+}
+
+// One thread per (unit, lane, step): one code word, and for lanes c < 2 one metadata word.
+__global__ void int4_pack_sparse24_kernel(const uint2* __restrict__ w, const uint8_t* __restrict__ codes,
+                                          const uint16_t* __restrict__ scales, uint32_t N, uint32_t K,
+                                          uint32_t* __restrict__ packed, uint32_t* __restrict__ pscales) {
+  const uint32_t G = K >> 7;
+  const uint64_t units = (uint64_t)(N >> 4) * G;
+  const uint64_t total = units * 128;
+  for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (uint64_t)gridDim.x * blockDim.x) {
+    const uint64_t unit = i >> 7;
+    const uint32_t lane = (uint32_t)(i >> 2) & 31u, s = (uint32_t)i & 3u;
+    const uint32_t g = lane >> 2, c = lane & 3u;
+    const uint32_t nt = (uint32_t)(unit / G), gi = (uint32_t)(unit - (uint64_t)nt * G);
+    auto kept_code = [&](uint32_t row, uint32_t run, uint32_t q) {   // q-th kept code of a run
+      const uint32_t k0 = 128 * gi + 4 * run;
+      const uint32_t m = run_meta(__ldg(w + ((size_t)row * K + k0) / 4));
+      const uint32_t k = k0 + (q ? (m >> 2) : (m & 3u));
+      return (uint32_t)(__ldg(codes + (size_t)row * (K / 2) + k / 2) >> (4 * (k & 1u))) & 0xFu;
+    };
+    uint32_t word = 0;
+#pragma unroll
+    for (int reg = 0; reg < 4; ++reg) {
+      const uint32_t row = 16 * nt + g + ((reg & 1) ? 8u : 0u);
+      const uint32_t kc = 2 * c + ((reg & 2) ? 8u : 0u);   // compressed k of the register's low half
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t kk = kc + h;
+        word |= kept_code(row, sparse_run(s, kk >> 1), kk & 1u) << (4 * (reg + 4 * h));
+      }
+    }
+    uint32_t* u = packed + unit * 192;                       // 768 bytes per unit
+    u[4 * lane + s] = word;
+    if (c < 2) {
+      uint32_t m = 0;
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        const uint32_t row = 16 * nt + g + 8 * (n >> 2);
+        const uint32_t run = sparse_run(s, 4 * c + (n & 3));
+        m |= run_meta(__ldg(w + ((size_t)row * K + 128 * gi + 4 * run) / 4)) << (4 * n);
+      }
+      u[128 + 4 * (2 * g + c) + s] = m;
+    }
+    if (lane < 8 && s == 0) {                                // word g: rows g (low) and g + 8 (high)
+      const uint32_t lo = __ldg(scales + (size_t)(16 * nt + lane) * G + gi);
+      const uint32_t hi = __ldg(scales + (size_t)(16 * nt + lane + 8) * G + gi);
+      pscales[unit * 8 + lane] = lo | (hi << 16);
+    }
+  }
+}
+
+}  // namespace nvq

@@ -85,11 +85,11 @@ constexpr int64_t kMaxDim = (int64_t)1 << 31;
 // tiles.  Batch rows are handled 8 * NT8 at a time.
 constexpr int kMaxDevices = 64;
 
-template <int NT8>
+template <int NT8, bool SPARSE = false>
 nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* y, int64_t M, int64_t N, int64_t K,
                         cudaStream_t stream) {
-  using C = nvq::w4a16::Cfg<NT8>;
-  auto fn = nvq::w4a16::w4a16_kernel<NT8>;
+  using C = nvq::w4a16::Cfg<NT8, SPARSE>;
+  auto fn = nvq::w4a16::w4a16_kernel<NT8, SPARSE>;
   static int max_clusters[kMaxDevices] = {};     // 0: not queried yet on that device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -480,6 +480,43 @@ nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const voi
   if (M <= 8) return launch_w4a16<1>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
   if (M <= 16) return launch_w4a16<2>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
   return launch_w4a16<4>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
+}
+
+// ------------------------------------------------------------------ 2:4 sparse INT4 decode
+nvq_status int4_pack_sparse24(const void* w_bf16, const uint8_t* codes, const void* scales_bf16, int64_t N,
+                              int64_t K, uint8_t* packed, void* packed_scales, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (N < 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "int4_pack_sparse24: bad sizes");
+  if (N % 16 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_pack_sparse24: need N % 16 == 0, K % 128 == 0");
+  if (N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_pack_sparse24: too large");
+  if (N == 0) return NVQ_OK;
+  if (!w_bf16 || !codes || !scales_bf16 || !packed || !packed_scales)
+    return fail(NVQ_ERR_INVALID_ARG, "int4_pack_sparse24: NULL pointer");
+  if (!aligned16(w_bf16) || !aligned16(codes) || !aligned16(scales_bf16) || !aligned16(packed) || !aligned16(packed_scales))
+    return fail(NVQ_ERR_MISALIGNED, "int4_pack_sparse24: pointer not 16-byte aligned");
+  const uint64_t threads = (uint64_t)(N / 16) * (uint64_t)(K / 128) * 128;
+  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>((threads + 255) / 256, (uint64_t)sm_count() * 16));
+  nvq::int4_pack_sparse24_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint2*>(w_bf16), codes,
+                                                           static_cast<const uint16_t*>(scales_bf16), (uint32_t)N,
+                                                           (uint32_t)K, reinterpret_cast<uint32_t*>(packed),
+                                                           static_cast<uint32_t*>(packed_scales));
+  return launch_status("int4_pack_sparse24_kernel");
+}
+
+nvq_status w4a16_sparse24_gemm(const void* x_bf16, const uint8_t* packed, const void* packed_scales, void* y_bf16,
+                               int64_t M, int64_t N, int64_t K, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "w4a16_sparse24_gemm: bad sizes");
+  if (N % 16 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_sparse24_gemm: need N % 16 == 0, K % 128 == 0");
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || (N / 16) * (K / 128) >= ((int64_t)1 << 32))
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_sparse24_gemm: too large");
+  if (M == 0) return NVQ_OK;
+  if (!x_bf16 || !packed || !packed_scales || !y_bf16) return fail(NVQ_ERR_INVALID_ARG, "w4a16_sparse24_gemm: NULL pointer");
+  if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(packed_scales) || !aligned16(y_bf16))
+    return fail(NVQ_ERR_MISALIGNED, "w4a16_sparse24_gemm: pointer not 16-byte aligned");
+  if (M <= 8) return launch_w4a16<1, true>(x_bf16, packed, packed_scales, y_bf16, M, N, K, stream);
+  if (M <= 16) return launch_w4a16<2, true>(x_bf16, packed, packed_scales, y_bf16, M, N, K, stream);
+  return launch_w4a16<4, true>(x_bf16, packed, packed_scales, y_bf16, M, N, K, stream);
 }
 
 // ------------------------------------------------------------------ phase dispatch

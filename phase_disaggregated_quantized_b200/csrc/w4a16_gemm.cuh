@@ -40,14 +40,20 @@ namespace w4a16 {
 
 constexpr int SG = 4;                        // groups per ring stage
 constexpr int CS = 2;                        // CTAs per cluster (74 such pairs fill 148 SMs)
-constexpr uint32_t GROUP_BYTES = 1024 + 32;  // codes + scales of one group
+// Bytes of one 16-row x 128-k group: codes (dense 1024; 2:4 sparse 512 of kept
+// codes + 256 of metadata) and 32 of scales.
+template <bool SPARSE>
+struct Unit {
+  static constexpr uint32_t CODE = SPARSE ? 768u : 1024u;
+  static constexpr uint32_t BYTES = CODE + 32u;
+};
 
-template <int NT8>
+template <int NT8, bool SPARSE = false>
 struct Cfg {
   static constexpr int W = NT8 == 1 ? 16 : 8;          // warps per CTA (register budget)
   static constexpr int D = NT8 == 1 ? 3 : 6;           // ring stages per warp
   static constexpr int THREADS = W * 32;
-  static constexpr int STAGE = SG * GROUP_BYTES;
+  static constexpr int STAGE = SG * Unit<SPARSE>::BYTES;
   static constexpr int RING = W * D * STAGE;
   static constexpr int TILEF = 128 * NT8;               // floats of one 16 x (8 NT8) partial tile
   static constexpr int BARS = RING;                      // W * D stage barriers
@@ -225,11 +231,65 @@ __device__ __forceinline__ void group_mma(const uint4 wa, const uint4 wb, const 
   }
 }
 
-template <int NT8>
-__global__ void __launch_bounds__(Cfg<NT8>::THREADS, 1) w4a16_kernel(
+// d += A * B for one m16n8k32 step with a 2:4-sparse A (compressed 16 x 16
+// values, metadata e from lanes c = 0, 1 of each quad).
+__device__ __forceinline__ void mma_sp_acc(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[4], uint32_t e) {
+  asm volatile(
+      "mma.sp::ordered_metadata.sync.aligned.m16n8k32.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9,%10,%11}, {%0,%1,%2,%3}, %12, 0x0;"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3]), "r"(e));
+}
+
+// One 2:4-sparse unit (16 rows x 128 k, 64 kept codes per row): four m16n8k32
+// steps; step s reads runs 8 s .. 8 s + 7 of the group, so lane (g, c) needs
+// activations k = 32 s + 16 (c / 2) + {0 .. 15}, of which words c % 2, 2 + c % 2,
+// 4 + c % 2, 6 + c % 2 feed its B fragment.  t0 / t1 receive the even / odd steps.
+template <int NT8, bool ONES>
+__device__ __forceinline__ void sparse_group(uint32_t unit, uint32_t lane, const uint4* const (&xrow)[NT8],
+                                             const bool (&live)[NT8], uint32_t gk, float (&t0)[NT8][4],
+                                             float (&t1)[NT8][4]) {
+  const uint32_t g = lane >> 2, c = lane & 3u, odd = c & 1u;
+  const uint4 wq = lds128(unit + lane * 16);
+  const uint4 mq = lds128(unit + 512 + (2 * g + odd) * 16);   // lanes c >= 2 load a copy the MMA ignores
+  const uint32_t wsw[4] = {wq.x, wq.y, wq.z, wq.w};
+  const uint32_t msw[4] = {mq.x, mq.y, mq.z, mq.w};
+  constexpr uint32_t kNeg136 = 0xC308C308u;
+  const uint32_t neg[4] = {kNeg136, kNeg136, kNeg136, kNeg136};
+#pragma unroll
+  for (int t = 0; t < NT8; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) t0[t][e] = t1[t][e] = 0.f;
+#pragma unroll
+  for (int st = 0; st < 4; ++st) {
+    uint32_t a[4];
+    word_to_frag(wsw[st], a);
+    if (!ONES) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = bf16x2_sub136(a[i]);
+    }
+#pragma unroll
+    for (int t = 0; t < NT8; ++t) {
+      uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
+      if (live[t]) {
+        const uint4* px = xrow[t] + gk * 16u + 4u * st + 2u * (c >> 1);
+        x0 = __ldg(px);
+        x1 = __ldg(px + 1);
+      }
+      const uint32_t b[4] = {odd ? x0.y : x0.x, odd ? x0.w : x0.z, odd ? x1.y : x1.x, odd ? x1.w : x1.z};
+      float (&d)[4] = (st & 1) ? t1[t] : t0[t];
+      mma_sp_acc(d, a, b, msw[st]);
+      if (ONES) mma_sp_acc(d, neg, b, msw[st]);
+    }
+  }
+}
+
+template <int NT8, bool SPARSE>
+__global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, 1) w4a16_kernel(
     const __nv_bfloat16* __restrict__ x, const uint8_t* __restrict__ pcodes, const uint8_t* __restrict__ pscales,
     __nv_bfloat16* __restrict__ y, uint32_t M, uint32_t N, uint32_t K) {
-  using C = Cfg<NT8>;
+  using C = Cfg<NT8, SPARSE>;
+  constexpr uint32_t UC = Unit<SPARSE>::CODE;
   constexpr int W = C::W, D = C::D;
   constexpr uint32_t MC = 8 * NT8, TILEF = C::TILEF;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -275,17 +335,17 @@ __global__ void __launch_bounds__(Cfg<NT8>::THREADS, 1) w4a16_kernel(
     if (nf > 0 && ok) {
       // Stages hold up to SG groups and never straddle a tile, so a stage's
       // groups share one tile and consecutive k-groups.
-      const uint8_t* wnext = pcodes + (size_t)f0 * 1024;
+      const uint8_t* wnext = pcodes + (size_t)f0 * UC;
       const uint8_t* snext = pscales + (size_t)f0 * 32;
       uint32_t irem = nf, ig = g_first, islot = cs;
       auto issue = [&]() {                    // lane 0: the next stage of this warp's range
         const uint32_t n = min(min(irem, (uint32_t)SG), G - ig);
         const uint32_t bar = bars + 8 * islot;
         const uint32_t dst = ring + islot * C::STAGE;
-        mbar_arrive_expect_tx(bar, n * GROUP_BYTES);
-        bulk_load_l2hint(dst, wnext, n * 1024u, bar, pol);
-        bulk_load_l2hint(dst + SG * 1024, snext, n * 32u, bar, pol);
-        wnext += n * 1024;
+        mbar_arrive_expect_tx(bar, n * Unit<SPARSE>::BYTES);
+        bulk_load_l2hint(dst, wnext, n * UC, bar, pol);
+        bulk_load_l2hint(dst + SG * UC, snext, n * 32u, bar, pol);
+        wnext += n * UC;
         snext += n * 32;
         irem -= n;
         ig = ig + n == G ? 0u : ig + n;
@@ -304,7 +364,7 @@ __global__ void __launch_bounds__(Cfg<NT8>::THREADS, 1) w4a16_kernel(
       for (int t = 0; t < NT8; ++t) {
         const uint32_t m = m0 + 8 * t + gl;
         live[t] = m < M;
-        xrow[t] = reinterpret_cast<const uint4*>(x + (size_t)(live[t] ? m : 0) * K + 32u * (lane & 3u));
+        xrow[t] = reinterpret_cast<const uint4*>(x + (size_t)(live[t] ? m : 0) * K + (SPARSE ? 0u : 32u * (lane & 3u)));
       }
       uint4 xa[NT8][4], xb[NT8][4];
 #pragma unroll
@@ -321,23 +381,27 @@ __global__ void __launch_bounds__(Cfg<NT8>::THREADS, 1) w4a16_kernel(
         if (!mbar_wait(bars + 8 * cs, phase)) { ok = false; break; }
         const uint32_t n = min(min(left, (uint32_t)SG), G - g);
         const uint32_t w_addr = ring + cs * C::STAGE + lane * 16;
-        const uint32_t s_addr = ring + cs * C::STAGE + SG * 1024 + gl * 4;
+        const uint32_t s_addr = ring + cs * C::STAGE + SG * UC + gl * 4;
 #pragma unroll
         for (int i = 0; i < SG; ++i) {
           if ((uint32_t)i < n) {
-            uint4 (&cur)[NT8][4] = (i & 1) ? xb : xa;
-            uint4 (&nxt)[NT8][4] = (i & 1) ? xa : xb;
-            const uint32_t gn = g + i + 1 == G ? 0u : g + i + 1;       // next group's k-block
-#pragma unroll
-            for (int t = 0; t < NT8; ++t)
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                if (live[t]) nxt[t][v] = __ldg(xrow[t] + gn * 16u + v);
-            const uint4 wa = lds128(w_addr + i * 1024);
-            const uint4 wb = lds128(w_addr + i * 1024 + 512);
-            const uint32_t scw = lds32(s_addr + i * 32);
             float t0[NT8][4], t1[NT8][4];
-            group_mma<NT8, C::ONES>(wa, wb, cur, t0, t1);
+            if constexpr (SPARSE) {
+              sparse_group<NT8, C::ONES>(ring + cs * C::STAGE + i * UC, lane, xrow, live, g + i, t0, t1);
+            } else {
+              uint4 (&cur)[NT8][4] = (i & 1) ? xb : xa;
+              uint4 (&nxt)[NT8][4] = (i & 1) ? xa : xb;
+              const uint32_t gn = g + i + 1 == G ? 0u : g + i + 1;     // next group's k-block
+#pragma unroll
+              for (int t = 0; t < NT8; ++t)
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                  if (live[t]) nxt[t][v] = __ldg(xrow[t] + gn * 16u + v);
+              const uint4 wa = lds128(w_addr + i * UC);
+              const uint4 wb = lds128(w_addr + i * UC + 512);
+              group_mma<NT8, C::ONES>(wa, wb, cur, t0, t1);
+            }
+            const uint32_t scw = lds32(s_addr + i * 32);
             const float s_lo = __uint_as_float(scw << 16), s_hi = __uint_as_float(scw & 0xFFFF0000u);
 #pragma unroll
             for (int t = 0; t < NT8; ++t) {
@@ -348,7 +412,7 @@ __global__ void __launch_bounds__(Cfg<NT8>::THREADS, 1) w4a16_kernel(
             }
           }
         }
-        if (n & 1) {                          // the next group's activations sit in xb
+        if (!SPARSE && (n & 1)) {             // the next group's activations sit in xb
 #pragma unroll
           for (int t = 0; t < NT8; ++t)
 #pragma unroll

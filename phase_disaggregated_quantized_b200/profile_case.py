@@ -32,6 +32,7 @@ def main():
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--N", type=int, default=0)
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--sparse", action="store_true", help="w4a16: the 2:4-sparse packed weights")
     ap.add_argument("--copies", type=int, default=1,
                     help="w4a16: cycle through this many weight copies (a total above L2 gives cold-cache reads)")
     a = ap.parse_args()
@@ -55,7 +56,10 @@ def main():
     elif a.op == "w4a16":
         w = synth.weights_cuda(a.N, a.K, seed=11, device=dev)
         codes, scales = nvq.int4_quantize(w)
-        packed = [nvq.int4_pack_weights(codes, scales, a.N, a.K) for _ in range(a.copies)]
+        if a.sparse:
+            packed = [nvq.int4_pack_sparse24(w, codes, scales) for _ in range(a.copies)]
+        else:
+            packed = [nvq.int4_pack_weights(codes, scales, a.N, a.K) for _ in range(a.copies)]
         y = torch.empty(a.M, a.N, dtype=torch.bfloat16, device=dev)
         ws = torch.empty(max(16, nvq.w4a16_workspace_bytes(a.M, a.N, a.K)), dtype=torch.uint8, device=dev)
         calls = [0]
@@ -63,8 +67,12 @@ def main():
         def run():
             pc, ps = packed[calls[0] % len(packed)]
             calls[0] += 1
-            nvq.w4a16_gemm(x, pc, ps, a.N, y=y, workspace=ws)
-        work = a.N * a.K / 2 + 2 * a.N * a.K / 128 + 2 * a.M * a.K + 2 * a.M * a.N
+            if a.sparse:
+                nvq.w4a16_sparse24_gemm(x, pc, ps, a.N, y=y)
+            else:
+                nvq.w4a16_gemm(x, pc, ps, a.N, y=y, workspace=ws)
+        wbytes = a.N * a.K * 3 / 8 if a.sparse else a.N * a.K / 2
+        work = wbytes + 2 * a.N * a.K / 128 + 2 * a.M * a.K + 2 * a.M * a.N
         unit = "GB/s"
     else:
         codes = torch.empty(a.M, a.K // 2, dtype=torch.uint8, device=dev)

@@ -338,6 +338,61 @@ def test_crossover_sweep_both_paths_sampled(M):
     assert ok, ("w4a16", M, worst)
 
 
+# ------------------------------------------------------------------ 2:4 sparse INT4 decode
+
+def gpu_sparse24(w_cpu):
+    N, K = w_cpu.shape
+    wd = w_cpu.cuda()
+    codes, scales = nvq.int4_quantize(wd)
+    p, ps = nvq.int4_pack_sparse24(wd, codes, scales)
+    nvq.check_device_error()
+    return p, ps
+
+
+@pytest.mark.parametrize("N,K", [(16, 128), (64, 512), (48, 384)])
+def test_sparse24_pack_bit_exact(N, K):
+    from oracle import sparse24 as osp
+    w = synth.weights(N, K, seed=N * 7 + K)
+    w[1, :8] = 0                                              # runs of zeros: ties everywhere
+    w[2, 4:8] = w[2, 4]                                       # four equal magnitudes
+    p, ps = gpu_sparse24(w)
+    u, meta, s_bits, _ = osp.quantize(bf16_to_f64(w))
+    op, ops = osp.pack(u, meta, s_bits)
+    np.testing.assert_array_equal(u8(p), op)
+    np.testing.assert_array_equal(u8(ps), ops)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (4, 512, 1024), (8, 1024, 256), (13, 272, 384), (16, 512, 512),
+                                   (32, 1024, 2048), (40, 256, 1024), (1, 16, 128)])
+def test_sparse24_decode_matches_oracle(M, N, K):
+    from oracle import sparse24 as osp
+    x = synth.activations(M, K, seed=M + 3 * K)
+    w = synth.weights(N, K, seed=N + 5)
+    p, ps = gpu_sparse24(w)
+    y = nvq.w4a16_sparse24_gemm(x.cuda(), p, ps, N)
+    nvq.check_device_error()
+    u, meta, s_bits, _ = osp.quantize(bf16_to_f64(w))
+    y_ref = osp.w4a16_ref(bf16_to_f64(x), u, meta, s_bits)
+    ok, worst = onv.within_tolerance(bf16_to_f64(y), y_ref)
+    assert ok, (M, N, K, worst)
+
+
+@pytest.mark.parametrize("layer", range(4))
+def test_sparse24_decode_qwen3_8b_full_size(layer):
+    from oracle import sparse24 as osp
+    name, K, N = synth.QWEN3_8B_LINEARS[layer]
+    w = synth.weights(N, K, seed=3100 + 10 * layer)
+    p, ps = gpu_sparse24(w)
+    u, meta, s_bits, _ = osp.quantize(bf16_to_f64(w))
+    for M in (1, 16):
+        x = synth.activations(M, K, seed=3200 + M + layer)
+        y = nvq.w4a16_sparse24_gemm(x.cuda(), p, ps, N)
+        nvq.check_device_error()
+        y_ref = osp.w4a16_ref(bf16_to_f64(x), u, meta, s_bits)
+        ok, worst = onv.within_tolerance(bf16_to_f64(y), y_ref)
+        assert ok, (name, M, worst)
+
+
 # ------------------------------------------------------------------ phase dispatch
 
 @pytest.mark.parametrize("M", [1, 8, 9, 40])
