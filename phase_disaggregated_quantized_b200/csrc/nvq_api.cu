@@ -96,11 +96,13 @@ nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* 
   if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm: cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(NVQ_ERR_CUDA, "w4a16_gemm: device index out of range");
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = nvq::w4a16::CS;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // may launch during the previous kernel's tail
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = stream;
@@ -119,6 +121,7 @@ nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* 
   const int64_t tiles = N / 16;
   const int64_t nclu = std::min<int64_t>(max_clusters[dev], tiles);
   cfg.gridDim = dim3((unsigned)(nclu * nvq::w4a16::CS), 1, 1);
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, fn, static_cast<const __nv_bfloat16*>(x), pc, static_cast<const uint8_t*>(ps),
                          static_cast<__nv_bfloat16*>(y), (uint32_t)M, (uint32_t)N, (uint32_t)K);
   if (e != cudaSuccess) return cuda_fail(e, "w4a16_kernel launch");

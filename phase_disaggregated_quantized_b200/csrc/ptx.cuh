@@ -84,6 +84,12 @@ __device__ __forceinline__ bool warp_mbar_wait(uint32_t bar, uint32_t parity) {
   return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0u;
 }
 
+// Programmatic dependent launch: wait until the grids this one depends on have
+// completed and their memory is visible (a no-op for a normal launch), and
+// allow the grids that depend on this one to start launching.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

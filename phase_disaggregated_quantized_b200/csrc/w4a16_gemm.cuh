@@ -320,6 +320,7 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, 1) w4a16_kernel(
     fence_mbar_init();
   }
   __syncwarp();
+  grid_dependency_wait();                      // before any global access (launched back to back)
   uint32_t cs = 0, phase = 0;                  // ring position of the next stage to consume
   uint32_t in_flight = 0;                      // lane 0: stages issued and not consumed
   bool ok = true;
@@ -459,6 +460,7 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, 1) w4a16_kernel(
       }
     }
 
+    if (pass + 1 == npass) grid_launch_dependents();   // the next kernel may start launching
     // ---- warps -> CTA: partial tiles summed in warp order through shared memory
     __syncthreads();                          // all rings idle: the slots may overlay them
     if (has0) put_tile<NT8>(wslots + (warp * 2 + 0) * TILEF + lane * 4 * NT8, p0);
