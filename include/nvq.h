@@ -187,18 +187,20 @@ nvq_status int4_quantize(const void* w_bf16, int64_t N, int64_t K, uint8_t* code
  * are regular and dequantize straight into tensor-core fragment order).  A
  * bijection: no byte is added or lost.
  *
- * Unit = 16 weight rows x one 128-wide group: 1024 code bytes at unit index
- * (n/16)*(K/128) + k/128.  Inside a unit, 32-bit word 128h + 4lane + jj (h in
- * {0,1}, lane = 4g + c in [0,32), jj in [0,4)) holds k16-step j = 4h + jj with
- * nibble p (bits 4p..4p+3) at (row, k-in-group); K is permuted inside the group
- * so that lane (g, c) covers k = 32c .. 32c+31:
+ * Unit = 32 weight rows x one 128-wide group: 2048 code bytes at unit index
+ * (n/32)*(K/128) + k/128; its rows are two 16-row tensor-core tiles tt = 0, 1.
+ * Inside a unit, 32-bit word 128q + 4lane + comp (q in [0,4), lane = 4g + c in
+ * [0,32), comp in [0,4)) holds k16-step j = 2q + comp/2 of tile tt = comp%2,
+ * with nibble p (bits 4p..4p+3) at (row in tile, k-in-group); K is permuted
+ * inside the group so that lane (g, c) covers k = 32c .. 32c+31:
  *   p=0 (g, 32c+4j)   p=4 (g, 32c+4j+1)   p=1 (g+8, 32c+4j)   p=5 (g+8, 32c+4j+1)
  *   p=2 (g, 32c+4j+2) p=6 (g, 32c+4j+3)   p=3 (g+8, 32c+4j+2) p=7 (g+8, 32c+4j+3)
- * Scales: 32 bytes per unit; 32-bit word g holds rows g (low) and g+8 (high).
+ * Scales: 64 bytes per unit; 32-bit word 2g + tt holds rows 16tt + g (low half)
+ * and 16tt + g + 8 (high half).
  *
  * codes [N, K/2] (as written by int4_quantize), scales_bf16 [N, K/128]
  * packed_codes N*K/2 bytes, packed_scales N*(K/128)*2 bytes, written.
- * Shape rules: N % 16 == 0, K % 128 == 0.
+ * Shape rules: N % 32 == 0, K % 128 == 0.
  * ------------------------------------------------------------------------ */
 nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int64_t N, int64_t K,
                              uint8_t* packed_codes, void* packed_scales, void* stream);
@@ -221,7 +223,7 @@ nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int6
  * workspace / workspace_bytes: unused (w4a16_workspace_bytes returns 0, the
  * partial sums stay on chip); kept so callers need not change.
  * Runs best for M <= 16; larger M is processed 32 rows per pass over W.
- * Shape rules: M >= 0, N % 16 == 0, K % 128 == 0.
+ * Shape rules: M >= 0, N % 32 == 0, K % 128 == 0.
  * ------------------------------------------------------------------------ */
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const void* packed_scales,
@@ -239,7 +241,8 @@ nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const voi
  * scales_bf16 are int4_quantize of the same W (a run's largest |w| is always
  * kept, so the group scales and the kept codes equal the dense ones).
  * packed: N*K*3/8 bytes (per 16-row x 128-k unit: 512 bytes of codes, 256 of
- * metadata); packed_scales: N*(K/128)*2 bytes, the layout of int4_pack_weights.
+ * metadata); packed_scales: N*(K/128)*2 bytes, 32 per unit, 32-bit word g
+ * holding rows g (low half) and g + 8 (high half) of the unit.
  *
  * w4a16_sparse24_gemm: Y = X (s (u - 8) at the kept positions, 0 elsewhere)^T,
  * with the arithmetic of w4a16_gemm (exact products, FP32 sums, group scale in
@@ -271,7 +274,7 @@ nvq_status w4a16_sparse24_gemm(const void* x_bf16, const uint8_t* packed, const 
  * workspace: nvq_linear_workspace_bytes(M, N, K, crossover_m) bytes, 16-byte
  * aligned (activation codes, scales, t and the quantizer's scratch), NULL when
  * that is 0.  Output y_bf16 [M, N] BF16, row stride N.
- * Shape rules: those of the chosen path (W4A16: N % 16 == 0, K % 128 == 0;
+ * Shape rules: those of the chosen path (W4A16: N % 32 == 0, K % 128 == 0;
  * W4A4: N % 8 == 0, K % 64 == 0).  Errors as the underlying calls.
  * ------------------------------------------------------------------------ */
 int64_t nvq_default_crossover_m(void);

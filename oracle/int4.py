@@ -117,19 +117,23 @@ def bytes_ratio_bf16_over_int4_g128(group: int = GROUP, scale_bytes: int = 2) ->
 # section of the MARLIN page: codes and group scales are permuted ahead of time
 # so each thread's loads are regular and land in tensor-core fragment order).
 #
-# The unit is a tile of 16 weight rows x one 128-wide group: 1024 code bytes
-# and 32 scale bytes, stored at unit index (n // 16) * (K / 128) + k // 128.
-# Inside a unit, 256 little-endian 32-bit words, word (h, lane, jj) at index
-# 128 h + 4 lane + jj holds k16-step j = 4 h + jj for lane = 4 g + c.  K is
-# permuted inside the group so that lane (g, c) covers k = 32c .. 32c+31:
-#   nibble p (bits 4p..4p+3), with r = row in tile, kk = k within the group:
+# The unit is a tile of 32 weight rows x one 128-wide group: 2048 code bytes
+# and 64 scale bytes, stored at unit index (n // 32) * (K / 128) + k // 128.
+# The 32 rows are two 16-row tensor-core tiles tt = 0, 1 (rows 16 tt .. 16 tt + 15).
+# Inside a unit, 512 little-endian 32-bit words; word (q, lane, comp) at index
+# 128 q + 4 lane + comp holds k16-step j = 2 q + comp // 2 of tile tt = comp % 2
+# for lane = 4 g + c.  K is permuted inside the group so that lane (g, c)
+# covers k = 32c .. 32c+31:
+#   nibble p (bits 4p..4p+3), with r = row in the 16-row tile, kk = k within the group:
 #     p=0: (g,   32c+4j)    p=4: (g,   32c+4j+1)
 #     p=1: (g+8, 32c+4j)    p=5: (g+8, 32c+4j+1)
 #     p=2: (g,   32c+4j+2)  p=6: (g,   32c+4j+3)
 #     p=3: (g+8, 32c+4j+2)  p=7: (g+8, 32c+4j+3)
-# Scale word g (g = 0..7) of a unit holds rows g (low half) and g+8 (high half).
+# Scale word 2 g + tt (g = 0..7) of a unit holds rows 16 tt + g (low half) and
+# 16 tt + g + 8 (high half).
 # ---------------------------------------------------------------------------
 
+UNIT_ROWS = 32
 _NIBBLE_ROW = np.array([0, 8, 0, 8, 0, 8, 0, 8])     # row offset added to g
 _NIBBLE_K = np.array([0, 0, 2, 2, 1, 1, 3, 3])       # k offset added to 32c+4j
 
@@ -139,18 +143,29 @@ def packed_code_index(N: int, K: int):
 
     Returns arrays n_idx, k_idx of shape [N*K/8, 8] indexed by packed word."""
     G = K // GROUP
-    units = (N // 16) * G
-    word = np.arange(256)
-    h, lane, jj = word // 128, (word // 4) % 32, word % 4
-    j = 4 * h + jj
+    units = (N // UNIT_ROWS) * G
+    word = np.arange(512)
+    q, lane, comp = word // 128, (word // 4) % 32, word % 4
+    j, tt = 2 * q + comp // 2, comp % 2
     g, c = lane // 4, lane % 4
-    r = g[:, None] + _NIBBLE_ROW[None, :]                          # [256, 8]
-    kk = (32 * c + 4 * j)[:, None] + _NIBBLE_K[None, :]            # [256, 8]
+    r = (16 * tt + g)[:, None] + _NIBBLE_ROW[None, :]              # [512, 8]
+    kk = (32 * c + 4 * j)[:, None] + _NIBBLE_K[None, :]            # [512, 8]
     unit = np.arange(units)
     nt, gi = unit // G, unit % G
-    n_idx = (16 * nt)[:, None, None] + r[None]                     # [units, 256, 8]
+    n_idx = (UNIT_ROWS * nt)[:, None, None] + r[None]              # [units, 512, 8]
     k_idx = (GROUP * gi)[:, None, None] + kk[None]
     return n_idx.reshape(-1, 8), k_idx.reshape(-1, 8)
+
+
+def _scale_rows(N: int, K: int):
+    """Row of every 16-bit scale slot: [units, 32] (slot 2 w + h of scale word w)."""
+    G = K // GROUP
+    unit = np.arange((N // UNIT_ROWS) * G)
+    nt = unit // G
+    w = np.arange(16)
+    g, tt = w // 2, w % 2
+    slot_row = np.stack([16 * tt + g, 16 * tt + g + 8], axis=1).reshape(-1)   # [32]
+    return (UNIT_ROWS * nt)[:, None] + slot_row[None, :], (unit % G)[:, None] + 0 * slot_row[None, :]
 
 
 def unpack_weights(packed_codes: np.ndarray, packed_scales: np.ndarray, N: int, K: int):
@@ -163,13 +178,10 @@ def unpack_weights(packed_codes: np.ndarray, packed_scales: np.ndarray, N: int, 
         u[n_idx[:, p], k_idx[:, p]] = (words >> np.uint32(4 * p)) & np.uint32(0xF)
     G = K // GROUP
     sw = np.frombuffer(np.ascontiguousarray(packed_scales, dtype=np.uint8).tobytes(),
-                       dtype="<u2").reshape((N // 16) * G, 16)
+                       dtype="<u2").reshape((N // UNIT_ROWS) * G, 32)
+    rows, gis = _scale_rows(N, K)
     s = np.zeros((N, G), dtype=np.uint16)
-    unit = np.arange((N // 16) * G)
-    nt, gi = unit // G, unit % G
-    for g in range(8):
-        s[16 * nt + g, gi] = sw[:, 2 * g]
-        s[16 * nt + g + 8, gi] = sw[:, 2 * g + 1]
+    s[rows, gis] = sw
     return u, s
 
 
@@ -180,11 +192,6 @@ def pack_weights(u: np.ndarray, s_bits: np.ndarray):
     words = np.zeros(n_idx.shape[0], dtype=np.uint32)
     for p in range(8):
         words |= u[n_idx[:, p], k_idx[:, p]].astype(np.uint32) << np.uint32(4 * p)
-    G = K // GROUP
-    unit = np.arange((N // 16) * G)
-    nt, gi = unit // G, unit % G
-    sw = np.zeros(((N // 16) * G, 16), dtype=np.uint16)
-    for g in range(8):
-        sw[:, 2 * g] = s_bits[16 * nt + g, gi]
-        sw[:, 2 * g + 1] = s_bits[16 * nt + g + 8, gi]
+    rows, gis = _scale_rows(N, K)
+    sw = s_bits[rows, gis].astype(np.uint16)
     return words.view(np.uint8).copy(), sw.reshape(-1).view(np.uint8).copy()

@@ -56,26 +56,29 @@ __global__ void __launch_bounds__(kInt4QuantThreads) int4_quantize_kernel(
   }
 }
 
-// One thread per 32-bit word of packed codes; the first N*K/2048*8 threads also
-// write one 32-bit scale word each.
+// One thread per 32-bit word of packed codes; the first (N/32)*(K/128)*16
+// threads also write one 32-bit scale word each.  Dense unit = 32 rows x one
+// 128-k group (two 16-row MMA tiles tt): word 128 q + 4 lane + comp holds k16
+// step j = 2 q + comp / 2 of tile tt = comp % 2 for lane = 4 g + c; scale word
+// 2 g + tt holds rows 16 tt + g (low half) and 16 tt + g + 8 (high half).
 __global__ void int4_pack_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
                                  uint32_t N, uint32_t K, uint32_t* __restrict__ pcodes,
                                  uint32_t* __restrict__ pscales) {
   const uint32_t G = K >> 7;
   const uint64_t nwords = (uint64_t)N * K / 8;
-  const uint64_t nsw = (uint64_t)(N / 16) * G * 8;
+  const uint64_t nsw = (uint64_t)(N / 32) * G * 16;
   const uint32_t half_k = K >> 1;
   const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
   for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nwords; i += stride) {
-    const uint64_t unit = i >> 8;
-    const uint32_t word = (uint32_t)(i & 255u);
+    const uint64_t unit = i >> 9;
+    const uint32_t word = (uint32_t)(i & 511u);
     const uint32_t nt = (uint32_t)(unit / G), gi = (uint32_t)(unit % G);
-    const uint32_t h = word >> 7, lane = (word >> 2) & 31u, jj = word & 3u;
-    const uint32_t j = 4 * h + jj, g = lane >> 2, c = lane & 3u;
+    const uint32_t q = word >> 7, lane = (word >> 2) & 31u, comp = word & 3u;
+    const uint32_t j = 2 * q + (comp >> 1), tt = comp & 1u, g = lane >> 2, c = lane & 3u;
     uint32_t out = 0;
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
-      const uint32_t r = 16 * nt + g + ((p & 1) ? 8u : 0u);
+      const uint32_t r = 32 * nt + 16 * tt + g + ((p & 1) ? 8u : 0u);
       const uint32_t k = 128 * gi + 32 * c + 4 * j + ((p & 2) ? 2u : 0u) + ((p & 4) ? 1u : 0u);
       const uint32_t byte = codes[(size_t)r * half_k + (k >> 1)];
       out |= ((byte >> (4 * (k & 1))) & 0xFu) << (4 * p);
@@ -83,11 +86,12 @@ __global__ void int4_pack_kernel(const uint8_t* __restrict__ codes, const uint16
     pcodes[i] = out;
   }
   for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nsw; i += stride) {
-    const uint64_t unit = i >> 3;
-    const uint32_t g = (uint32_t)(i & 7u);
+    const uint64_t unit = i >> 4;
+    const uint32_t wi = (uint32_t)(i & 15u), g = wi >> 1, tt = wi & 1u;
     const uint32_t nt = (uint32_t)(unit / G), gi = (uint32_t)(unit % G);
-    const uint32_t lo = scales[(size_t)(16 * nt + g) * G + gi];
-    const uint32_t hi = scales[(size_t)(16 * nt + g + 8) * G + gi];
+    const uint32_t row = 32 * nt + 16 * tt + g;
+    const uint32_t lo = scales[(size_t)row * G + gi];
+    const uint32_t hi = scales[(size_t)(row + 8) * G + gi];
     pscales[i] = lo | (hi << 16);
   }
 }
@@ -103,7 +107,7 @@ namespace nvq {
 // the dense ones), written in the sparse decode kernel's order: per 16-row x
 // 128-k unit, 512 bytes of A-fragment code words (lane-major, 4 m16n8k32 steps
 // per lane) and 256 bytes of metadata words (lanes c = 0, 1), then the unit's
-// 32 bytes of scales as in int4_pack_kernel.
+// 32 bytes of scales (word g: rows g (low half) and g + 8 (high half)).
 
 // Kept positions (i0 < i1) of one run from its four bf16 values.
 __device__ __forceinline__ uint32_t run_meta(uint2 w4) {

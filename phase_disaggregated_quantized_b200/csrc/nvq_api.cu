@@ -81,8 +81,8 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uin
 constexpr int64_t kMaxDim = (int64_t)1 << 31;
 
 // Decode launch: a persistent grid of clusters of nvq::w4a16::CS CTAs, as many
-// as can be resident at once (one CTA per SM), never more clusters than 16-row
-// tiles.  Batch rows are handled 8 * NT8 at a time.
+// as can be resident at once (one CTA per SM), never more clusters than output
+// tiles (32 weight rows dense, 16 for 2:4 sparse).  Batch rows are handled 8 * NT8 at a time.
 constexpr int kMaxDevices = 64;
 
 template <int NT8, bool SPARSE = false>
@@ -118,7 +118,7 @@ nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* 
     if (n < 1) return fail(NVQ_ERR_CUDA, "w4a16_gemm: no cluster of the decode kernel fits on this GPU");
     max_clusters[dev] = n;
   }
-  const int64_t tiles = N / 16;
+  const int64_t tiles = N / nvq::w4a16::Unit<SPARSE>::ROWS;
   const int64_t nclu = std::min<int64_t>(max_clusters[dev], tiles);
   cfg.gridDim = dim3((unsigned)(nclu * nvq::w4a16::CS), 1, 1);
   cfg.numAttrs = 2;
@@ -443,8 +443,8 @@ nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int6
                              uint8_t* packed_codes, void* packed_scales, void* stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (N < 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "int4_pack_weights: bad sizes");
-  if (N % 16 != 0 || K % 128 != 0)
-    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_pack_weights: need N % 16 == 0, K % 128 == 0");
+  if (N % 32 != 0 || K % 128 != 0)
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_pack_weights: need N % 32 == 0, K % 128 == 0");
   if (N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_pack_weights: too large");
   if (N == 0) return NVQ_OK;
   if (!codes || !scales_bf16 || !packed_codes || !packed_scales)
@@ -473,8 +473,8 @@ nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const voi
   (void)workspace_bytes;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "w4a16_gemm: bad sizes");
-  if (N % 16 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_gemm: need N % 16 == 0, K % 128 == 0");
-  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || (N / 16) * (K / 128) >= ((int64_t)1 << 32))
+  if (N % 32 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_gemm: need N % 32 == 0, K % 128 == 0");
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || (N / 32) * (K / 128) >= ((int64_t)1 << 32))
     return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_gemm: too large");
   if (M == 0) return NVQ_OK;
   if (!x_bf16 || !packed_codes || !packed_scales || !y_bf16) return fail(NVQ_ERR_INVALID_ARG, "w4a16_gemm: NULL pointer");

@@ -79,10 +79,11 @@ def test_gemm_rejects_bad_arguments(L):
 
 def test_int4_calls_reject_bad_arguments(L):
     assert L.int4_quantize(_vp(FAKE), 16, 100, _vp(FAKE), _vp(FAKE), None) == 2
-    assert L.int4_pack_weights(_vp(FAKE), _vp(FAKE), 24, 128, _vp(FAKE), _vp(FAKE), None) == 2   # N % 16
+    assert L.int4_pack_weights(_vp(FAKE), _vp(FAKE), 48, 128, _vp(FAKE), _vp(FAKE), None) == 2   # N % 32
     assert L.int4_pack_weights(_vp(ODD), _vp(FAKE), 32, 128, _vp(FAKE), _vp(FAKE), None) == 3
     w = L.w4a16_gemm
     assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 24, 128, None, 0, None) == 2
+    assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 48, 128, None, 0, None) == 2     # N % 32
     assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(ODD), 4, 256, 4096, None, 0, None) == 3    # y misaligned
     assert w(_vp(FAKE), _vp(FAKE), None, _vp(FAKE), 4, 256, 4096, None, 0, None) == 1         # NULL scales
 
@@ -130,8 +131,8 @@ def test_phase_dispatch_host_rules(L):
              _vp(FAKE), _vp(ODD), 1 << 30, None) == 3
     assert f(_vp(FAKE), 4096, 256, 4100, _vp(FAKE), _vp(FAKE), _vp(FAKE), None, None, -1,
              _vp(FAKE), _vp(FAKE), 1 << 30, None) == 2
-    # W4A16 side keeps its own shape rules (N % 16)
-    assert f(_vp(FAKE), 1, 24, 4096, None, None, None, _vp(FAKE), _vp(FAKE), -1,
+    # W4A16 side keeps its own shape rules (N % 32)
+    assert f(_vp(FAKE), 1, 48, 4096, None, None, None, _vp(FAKE), _vp(FAKE), -1,
              _vp(FAKE), None, 0, None) == 2
 
 

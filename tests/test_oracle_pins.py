@@ -318,16 +318,21 @@ def test_int4_reorder_is_bijection_and_hand_slots():
     u2, s2 = int4.unpack_weights(pc, ps, N, K)
     assert np.array_equal(u, u2) and np.array_equal(s, s2)
     words = pc.view("<u4")
-    # unit 0, word 0 (lane 0, j 0): nibbles (0,0) (8,0) (0,2) (8,2) (0,1) (8,1) (0,3) (8,3)
+    # unit 0, word 0 (lane 0, j 0, tile 0): nibbles (0,0) (8,0) (0,2) (8,2) (0,1) (8,1) (0,3) (8,3)
     want = [u[0, 0], u[8, 0], u[0, 2], u[8, 2], u[0, 1], u[8, 1], u[0, 3], u[8, 3]]
     assert [(int(words[0]) >> (4 * p)) & 15 for p in range(8)] == [int(v) for v in want]
-    # lane 5 (g=1, c=1), j = 6 -> word 128 + 4*5 + 2, nibble 0 = (1, 32*1 + 4*6), nibble 7 = (9, 59)
-    assert (int(words[128 + 22]) & 15) == u[1, 56]
-    assert (int(words[128 + 22]) >> 28) == u[9, 59]
-    # unit 1 = tile 0, group 1: its word 0 nibble 0 is (0, 128)
-    assert (int(words[256]) & 15) == u[0, 128]
+    # word 1 = lane 0, j 0, tile 1 (rows 16..31): nibble 0 = (16, 0), nibble 7 = (24, 3)
+    assert (int(words[1]) & 15) == u[16, 0] and (int(words[1]) >> 28) == u[24, 3]
+    # lane 5 (g=1, c=1), j = 6, tile 0 -> word 128*3 + 4*5 + 0: nibble 0 = (1, 32*1 + 4*6), nibble 7 = (9, 59)
+    assert (int(words[404]) & 15) == u[1, 56]
+    assert (int(words[404]) >> 28) == u[9, 59]
+    # lane 5, j = 7, tile 1 -> word 384 + 20 + 3: nibble 0 = (17, 60), nibble 7 = (25, 63)
+    assert (int(words[407]) & 15) == u[17, 60] and (int(words[407]) >> 28) == u[25, 63]
+    # unit 1 = rows 0..31, group 1: its word 0 nibble 0 is (0, 128)
+    assert (int(words[512]) & 15) == u[0, 128]
     sw = ps.view("<u2")
-    assert sw[0] == s[0, 0] and sw[1] == s[8, 0] and sw[2] == s[1, 0] and sw[16] == s[0, 1]
+    assert sw[0] == s[0, 0] and sw[1] == s[8, 0] and sw[2] == s[16, 0] and sw[3] == s[24, 0]
+    assert sw[4] == s[1, 0] and sw[32] == s[0, 1]
 
 
 def test_int4_power_of_two_scale_is_exact_integer_dot():
