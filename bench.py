@@ -297,7 +297,11 @@ def run_gpu(args):
     ev = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
     q_ev = [(ev(), ev()) for _ in pre]
     g_ev = [(ev(), ev()) for _ in pre]
-    d_ev = [(ev(), ev()) for _ in DECODE_BATCHES]     # one timed region per batch size
+    # Decode is timed as two contiguous blocks (M <= 16, then M = 32): an event
+    # node between kernels ends programmatic dependent launch there, so timing
+    # each batch size separately would serialise calls a decode loop runs back
+    # to back.  Per-batch figures come from separate graphs (per_batch_decode).
+    d_ev = [(ev(), ev()), (ev(), ev())]
     pre_ev = (ev(), ev())
 
     def step():
@@ -312,10 +316,10 @@ def run_gpu(args):
                                 stream=stream)
             gb.record(stream)
         pre_ev[1].record(stream)
-        for M, (da, db) in zip(DECODE_BATCHES, d_ev):
+        for blk, (da, db) in enumerate(d_ev):
             da.record(stream)
             for D in dec:
-                if D["M"] == M:
+                if (D["M"] <= 16) == (blk == 0):
                     nvq.w4a16_gemm(D["x"], D["pc"], D["ps"], D["N"], y=D["y"], workspace=D["ws"], stream=stream)
             db.record(stream)
 
@@ -335,7 +339,7 @@ def run_gpu(args):
     t_start, t_end = ev(), ev()
     q_ms = [0.0] * len(pre)
     g_ms = [0.0] * len(pre)
-    d_ms = [0.0] * len(DECODE_BATCHES)
+    d_ms = [0.0] * len(d_ev)
     pre_ms = 0.0
     if world > 1:
         dist.barrier()
@@ -349,7 +353,7 @@ def run_gpu(args):
             for j in range(len(pre)):
                 q_ms[j] += q_ev[j][0].elapsed_time(q_ev[j][1])
                 g_ms[j] += g_ev[j][0].elapsed_time(g_ev[j][1])
-            for j in range(len(DECODE_BATCHES)):
+            for j in range(len(d_ev)):
                 d_ms[j] += d_ev[j][0].elapsed_time(d_ev[j][1])
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -368,16 +372,9 @@ def run_gpu(args):
         M, K, N = D["M"], D["K"], D["N"]
         return N * K / 2 + 2 * N * K / 128 + 2 * M * K + 2 * M * N
 
-    per_batch = {}
-    dec_b = dec_s = 0.0
-    for mi, M in enumerate(DECODE_BATCHES):
-        js = [j for j, D in enumerate(dec) if D["M"] == M]
-        b = sum(dec_bytes(dec[j]) for j in js)
-        s = d_ms[mi] / 1e3 / K_steps
-        per_batch[str(M)] = {"GB/s": b / s / 1e9, "us_per_call": 1e6 * s / len(js)}
-        if M <= 16:
-            dec_b += b
-            dec_s += s
+    dec_b = sum(dec_bytes(D) for D in dec if D["M"] <= 16)
+    dec_s = d_ms[0] / 1e3 / K_steps
+    per_batch = per_batch_decode(torch, nvq, dec, dec_w, stream, dec_bytes)
 
     peaks, peaks_kind = load_peaks()
     fp4_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP4_OVER_BF16
@@ -436,6 +433,40 @@ def run_gpu(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def per_batch_decode(torch, nvq, dec, dec_w, stream, dec_bytes, reps: int = 20):
+    """Per batch size: the four decode layers run back to back, cycling through
+    all weight copies (about 0.5 GB, so every weight byte comes from HBM), one
+    captured graph per batch size."""
+    out = {}
+    for M in DECODE_BATCHES:
+        calls = []
+        for copy in dec_w:
+            for D in dec:
+                if D["M"] == M:
+                    pc, ps = copy[D["layer"]]
+                    calls.append((D, pc, ps))
+        def run():
+            for D, pc, ps in calls:
+                nvq.w4a16_gemm(D["x"], pc, ps, D["N"], y=D["y"], workspace=D["ws"], stream=stream)
+        run()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run()
+        g.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        s = a.elapsed_time(b) / 1e3 / reps
+        by = sum(dec_bytes(D) for D, _, _ in calls)
+        out[str(M)] = {"GB/s": by / s / 1e9, "us_per_call": 1e6 * s / len(calls)}
+        del g
+    return out
 
 
 def measure_e2e(torch, nvq, pre, stream, steps: int):

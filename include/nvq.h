@@ -223,6 +223,12 @@ nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int6
  * workspace / workspace_bytes: unused (w4a16_workspace_bytes returns 0, the
  * partial sums stay on chip); kept so callers need not change.
  * Runs best for M <= 16; larger M is processed 32 rows per pass over W.
+ * Launched with programmatic dependent launch: the call may begin while the
+ * preceding kernel on the stream is still finishing, and it starts streaming
+ * the packed weights before waiting for that kernel (x and y are touched only
+ * after the wait).  So the packed weights must not be written by the kernel
+ * immediately before it when that kernel lets dependents launch early; no
+ * kernel of this library that writes them does, nor does an ordinary copy.
  * Shape rules: M >= 0, N % 32 == 0, K % 128 == 0.
  * ------------------------------------------------------------------------ */
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
