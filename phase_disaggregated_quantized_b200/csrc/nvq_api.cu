@@ -524,9 +524,9 @@ nvq_status w4a16_sparse24_gemm(const void* x_bf16, const uint8_t* packed, const 
 
 // ------------------------------------------------------------------ phase dispatch
 // Largest M at which W4A16 beat quantize + W4A4 on B200 for K = 4096, N = 24576
-// with weights read from HBM (profile_case --op crossover: 24.8 vs 30.2 us at
-// M = 8, 36.6 vs 29.2 us at M = 16).
-constexpr int64_t kDefaultCrossoverM = 8;
+// with weights read from HBM (profile_case --op crossover: 25.1 vs 28.9 us at
+// M = 16, 39.9 vs 30.0 us at M = 32).
+constexpr int64_t kDefaultCrossoverM = 16;
 
 int64_t nvq_default_crossover_m(void) { return kDefaultCrossoverM; }
 
