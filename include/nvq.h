@@ -213,7 +213,7 @@ nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int6
  *
  *   Y[m, n] = bf16_RNE( sum_g s[n, g] * sum_{k in g} x[m, k] * (u[n, k] - 8) )
  * with the inner sums accumulated in FP32 by the tensor cores and the group
- * scale applied in FP32.  All products are exact; for M <= 8 the inner sum is
+ * scale applied in FP32.  All products are exact; for M <= 16 the inner sum is
  * formed as sum x * (128 + u) + sum x * (-136), equal up to FP32 rounding.
  * Group sums are added in an order fixed by the shapes and the GPU's SM count,
  * so repeated calls give identical results.

@@ -23,7 +23,7 @@
 // k16 step j uses k = 32c + 4j + {0..3}: its 64-byte activation run feeds all
 // eight steps of both tiles of a dense unit.  Nibbles become bf16 (128 + u)
 // through the exponent bits.  The -136 offset (u - 8 = (128 + u) - 136) is
-// either subtracted in bf16 (exact) or, for one batch tile, formed once per
+// either subtracted in bf16 (exact) or, for up to two batch tiles, formed once per
 // unit as the chain -136 * sum(x) on the tensor core and passed as the C input
 // of both tiles' first MMA, so it costs no ALU work at all.  Each group's FP32
 // sum is scaled by the group's BF16 scale in FP32.
@@ -69,7 +69,7 @@ struct Cfg {
   static constexpr int XSLOT = (BARS + W * D * 8 + 15) / 16 * 16;   // 2 receive slots (pass parity)
   static constexpr int XBARS = XSLOT + 2 * TILEF * 4;    // receive-full [2], slot-free [2] barriers
   static constexpr int SMEM = XBARS + 32;
-  static constexpr bool ONES = NT8 == 1;                 // -136 x through the tensor core
+  static constexpr bool ONES = NT8 <= 2;                 // -136 x through the tensor core
   static constexpr bool XDB = NT8 <= 2;                  // activations double-buffered one unit ahead
   static_assert(STAGE % 16 == 0 && (SG * U::CODE) % 16 == 0, "bulk-copy alignment");
   static_assert(W * 2 * TILEF * 4 <= RING, "warp partial tiles overlay the ring");
