@@ -15,7 +15,8 @@
 //                scale atoms (A: 4, B: 2 row-atoms x 4) as plain bulk copies.
 //   warp 1       MMA issuer: per k-stage one wait for the stage's data and one
 //                for its scales in TMEM, four tcgen05.mma.kind::mxf4nvf4
-//                .block_scale.block16 (128 x 256 x 64), two commits.
+//                .block_scale.block16 (128 x 256 x 64), one commit (it frees the
+//                stage's operands and, two stages later, its scale slot).
 //   warps 2..9   epilogue, two warps per TMEM sub-partition, each draining one
 //                64-column chunk after another (tcgen05.ld), scaling by t_x t_w,
 //                rounding to bf16 and TMA-storing its own 32 rows x 64 columns
@@ -62,8 +63,8 @@ constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
 constexpr int OFF_SFA = OFF_C + EPI_WARPS * C_BYTES;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
 constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
-// full[S], empty[S], acc_full[2], acc_empty[2], overlap_free, sf_full[2], sf_free[2], drain
-constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 1 + 2 * SF_SLOTS + 1;
+// full[S], empty[S], acc_full[2], acc_empty[2], overlap_free, sf_full[2], drain
+constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 1 + SF_SLOTS + 1;
 constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;    // + slack for 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "smem budget");
@@ -212,8 +213,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
   const uint32_t bar_acc_empty = bar_acc_full + 16;           // + 8 b
   const uint32_t bar_overlap = bar_acc_empty + 16;
   const uint32_t bar_sf_full = bar_overlap + 8;               // + 8 slot
-  const uint32_t bar_sf_free = bar_sf_full + 8 * SF_SLOTS;    // + 8 slot
-  const uint32_t bar_drain = bar_sf_free + 8 * SF_SLOTS;
+  const uint32_t bar_drain = bar_sf_full + 8 * SF_SLOTS;
   uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(smem + OFF_TMEM_PTR);
 
   if (threadIdx.x == 0) {
@@ -228,7 +228,6 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     mbar_init(bar_overlap, EPI_WARPS);
     for (uint32_t k = 0; k < SF_SLOTS; ++k) {
       mbar_init(bar_sf_full + 8 * k, 4);                      // one arrive per scale-writer warp
-      mbar_init(bar_sf_free + 8 * k, 1);                      // one commit per k-stage from the MMA thread
     }
     mbar_init(bar_drain, 1);
     fence_mbar_init();
@@ -307,8 +306,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           const uint32_t natoms = min(4u, p.k_atoms - 4 * ks);
           for (uint32_t j = 0; j < natoms; ++j)     // 32 bytes (64 FP4 elements) per k step
             tc_mma_nvf4(d_tmem, ad + 2 * j, bd + 2 * j, IDESC, sf + 4 * j, sf + 16 + 8 * j, (ks | j) != 0u);
-          tc_commit(bar_empty + 8 * stage);
-          tc_commit(bar_sf_free + 8 * slot);
+          tc_commit(bar_empty + 8 * stage);                    // also frees this stage's scale slot
         }
         __syncwarp();
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -328,11 +326,19 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     // ------------------------------------------------------------ scale writers
     const uint32_t q = warp & 3u;                             // TMEM sub-partition of this warp
     const uint32_t lane_base = (q * 32u) << 16;
-    uint32_t stage = 0, phase = 0, slot = 0, slot_phase = 0;
+    uint32_t stage = 0, phase = 0, slot = 0;
+    // A scale slot is free once the MMAs of the k-stage that used it (SF_SLOTS
+    // k-stages back) have completed, i.e. once that stage's empty barrier has
+    // fired: one commit per k-stage serves the TMA producer and these warps
+    // (a tcgen05.commit costs the MMA thread about as much as an MMA).
+    uint32_t lag_stage = 0, lag_phase = 0, kg = 0;
     bool ok = true;
     for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      for (uint32_t ks = 0; ks < p.num_k_stages; ++ks) {
-        if (!(ok = warp_mbar_wait(bar_sf_free + 8 * slot, slot_phase ^ 1))) break;   // MMAs two stages back done
+      for (uint32_t ks = 0; ks < p.num_k_stages; ++ks, ++kg) {
+        if (kg >= SF_SLOTS) {
+          if (!(ok = warp_mbar_wait(bar_empty + 8 * lag_stage, lag_phase))) break;
+          if (++lag_stage == STAGES) { lag_stage = 0; lag_phase ^= 1; }
+        }
         if (!(ok = warp_mbar_wait(bar_full + 8 * stage, phase))) break;
         tc_fence_after();
         const uint8_t* sfa = smem + OFF_SFA + stage * SFA_BYTES + 16 * lane;
@@ -355,7 +361,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_sf_full + 8 * slot);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
-        if (++slot == SF_SLOTS) { slot = 0; slot_phase ^= 1; }
+        if (++slot == SF_SLOTS) slot = 0;
       }
     }
   } else {
