@@ -63,8 +63,8 @@ constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
 constexpr int OFF_SFA = OFF_C + EPI_WARPS * C_BYTES;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
 constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
-// full[S], empty[S], acc_full[2], acc_empty[2], overlap_free, sf_full[2], drain
-constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 1 + SF_SLOTS + 1;
+// full[S], empty[S], acc_full[2], acc_empty[2], overlap_free, sf_full[2], drain, scales_in[S]
+constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 1 + SF_SLOTS + 1 + STAGES;
 constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;    // + slack for 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "smem budget");
@@ -214,12 +214,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
   const uint32_t bar_overlap = bar_acc_empty + 16;
   const uint32_t bar_sf_full = bar_overlap + 8;               // + 8 slot
   const uint32_t bar_drain = bar_sf_full + 8 * SF_SLOTS;
+  const uint32_t bar_sc_in = bar_drain + 8;                   // + 8 s: the stage's scale atoms landed
   uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(smem + OFF_TMEM_PTR);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_sc_in + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_acc_full + 8 * b, 1);
@@ -259,16 +261,19 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         for (uint32_t ks = 0; ks < p.num_k_stages; ++ks) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
           const uint32_t natoms = min(4u, p.k_atoms - 4 * ks);
-          const uint32_t bytes = A_BYTES + B_BYTES + natoms * 512u * (1u + nb_atoms);
-          const uint32_t fb = bar_full + 8 * stage;
-          mbar_arrive_expect_tx(fb, bytes);
-          tma_load_2d(sbase + OFF_A + stage * A_BYTES, &tmap_a, fb, (int)(ks * BKB), (int)(mt * BM), pol);
-          tma_load_2d(sbase + OFF_B + stage * B_BYTES, &tmap_b, fb, (int)(ks * BKB), (int)(nt * BN), pol);
+          // The scale atoms complete on a barrier of their own and go first, so
+          // the scale writers can move them into TMEM while the operands land.
+          const uint32_t sb = bar_sc_in + 8 * stage;
+          mbar_arrive_expect_tx(sb, natoms * 512u * (1u + nb_atoms));
           bulk_load(sbase + OFF_SFA + stage * SFA_BYTES,
-                    p.x_scales + ((size_t)mt * p.k_atoms + 4 * ks) * 512u, natoms * 512u, fb);
+                    p.x_scales + ((size_t)mt * p.k_atoms + 4 * ks) * 512u, natoms * 512u, sb);
           for (uint32_t a = 0; a < nb_atoms; ++a)
             bulk_load(sbase + OFF_SFB + stage * SFB_BYTES + a * 2048u,
-                      p.w_scales + ((size_t)(2 * nt + a) * p.k_atoms + 4 * ks) * 512u, natoms * 512u, fb);
+                      p.w_scales + ((size_t)(2 * nt + a) * p.k_atoms + 4 * ks) * 512u, natoms * 512u, sb);
+          const uint32_t fb = bar_full + 8 * stage;
+          mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+          tma_load_2d(sbase + OFF_A + stage * A_BYTES, &tmap_a, fb, (int)(ks * BKB), (int)(mt * BM), pol);
+          tma_load_2d(sbase + OFF_B + stage * B_BYTES, &tmap_b, fb, (int)(ks * BKB), (int)(nt * BN), pol);
           pending |= 1u << stage;
           pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -276,7 +281,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       }
       // Let every copy issued into shared memory land before the CTA exits.
       for (int s2 = 0; s2 < STAGES; ++s2)
-        if (pending & (1u << s2)) mbar_wait_drain(bar_full + 8 * s2, (pending_parity >> s2) & 1u, 200000000ull);
+        if (pending & (1u << s2)) {
+          mbar_wait_drain(bar_sc_in + 8 * s2, (pending_parity >> s2) & 1u, 200000000ull);
+          mbar_wait_drain(bar_full + 8 * s2, (pending_parity >> s2) & 1u, 200000000ull);
+        }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -339,22 +347,37 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           if (!(ok = warp_mbar_wait(bar_empty + 8 * lag_stage, lag_phase))) break;
           if (++lag_stage == STAGES) { lag_stage = 0; lag_phase ^= 1; }
         }
-        if (!(ok = warp_mbar_wait(bar_full + 8 * stage, phase))) break;
+        if (!(ok = warp_mbar_wait(bar_sc_in + 8 * stage, phase))) break;   // this stage's scale atoms
         tc_fence_after();
         const uint8_t* sfa = smem + OFF_SFA + stage * SFA_BYTES + 16 * lane;
         const uint8_t* sfb = smem + OFF_SFB + stage * SFB_BYTES + 16 * lane;
         const uint32_t col = lane_base + tmem_base + SF_COL0 + SF_SLOT_COLS * slot;
         const uint32_t natoms = min(4u, p.k_atoms - 4 * ks);
-        for (uint32_t j = 0; j < natoms; ++j) {
-          // Atom row `lane` holds rows lane, lane+32, lane+64, lane+96 (4 bytes each);
-          // column c gets rows 32c + lane, as tcgen05.cp .32x128b.warpx4 would place them.
-          const uint4 a = *reinterpret_cast<const uint4*>(sfa + 512 * j);
-          const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j);
-          const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + 2048 + 512 * j);
-          const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-          const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-          tc_st_32x32b_x4(col + 4 * j, aw);
-          tc_st_32x32b_x8(col + 16 + 8 * j, bw);
+        // Atom row `lane` holds rows lane, lane+32, lane+64, lane+96 (4 bytes each);
+        // column c gets rows 32c + lane, as tcgen05.cp .32x128b.warpx4 would place them.
+        if (natoms == 4u) {                   // whole stage: two wide TMEM stores
+          uint32_t aw[16], bw[32];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 a = *reinterpret_cast<const uint4*>(sfa + 512 * j);
+            const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j);
+            const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + 2048 + 512 * j);
+            aw[4 * j] = a.x; aw[4 * j + 1] = a.y; aw[4 * j + 2] = a.z; aw[4 * j + 3] = a.w;
+            bw[8 * j] = b0.x; bw[8 * j + 1] = b0.y; bw[8 * j + 2] = b0.z; bw[8 * j + 3] = b0.w;
+            bw[8 * j + 4] = b1.x; bw[8 * j + 5] = b1.y; bw[8 * j + 6] = b1.z; bw[8 * j + 7] = b1.w;
+          }
+          tc_st_32x32b_x16(col, aw);
+          tc_st_32x32b_x32(col + 16, bw);
+        } else {
+          for (uint32_t j = 0; j < natoms; ++j) {
+            const uint4 a = *reinterpret_cast<const uint4*>(sfa + 512 * j);
+            const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * j);
+            const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + 2048 + 512 * j);
+            const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+            const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            tc_st_32x32b_x4(col + 4 * j, aw);
+            tc_st_32x32b_x8(col + 16 + 8 * j, bw);
+          }
         }
         tc_wait_st();
         tc_fence_before();
