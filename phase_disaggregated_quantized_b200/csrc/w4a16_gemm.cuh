@@ -57,7 +57,7 @@ struct Unit {
 template <int NT8, bool SPARSE = false>
 struct Cfg {
   using U = Unit<SPARSE>;
-  static constexpr int W = NT8 == 1 ? 16 : 8;          // warps per CTA (register budget)
+  static constexpr int W = 8;                          // warps per CTA (two CTAs per SM)
   static constexpr int SG = SPARSE ? 4 : 2;            // units per ring stage
   static constexpr int D = NT8 == 1 ? 3 : 6;           // ring stages per warp
   static constexpr int THREADS = W * 32;
