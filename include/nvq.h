@@ -246,14 +246,15 @@ nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const voi
  * m16n8k32 sparse MMA, with their 2-bit positions as MMA metadata.  codes and
  * scales_bf16 are int4_quantize of the same W (a run's largest |w| is always
  * kept, so the group scales and the kept codes equal the dense ones).
- * packed: N*K*3/8 bytes (per 16-row x 128-k unit: 512 bytes of codes, 256 of
- * metadata); packed_scales: N*(K/128)*2 bytes, 32 per unit, 32-bit word g
- * holding rows g (low half) and g + 8 (high half) of the unit.
+ * packed: N*K*3/8 bytes (per 32-row x 128-k unit, unit index
+ * (n/32)*(K/128) + k/128: two 16-row tiles tt, each 512 bytes of codes then
+ * 256 of metadata); packed_scales: N*(K/128)*2 bytes, 64 per unit, 32-bit word
+ * 2g + tt holding rows 16tt + g (low half) and 16tt + g + 8 (high half).
  *
  * w4a16_sparse24_gemm: Y = X (s (u - 8) at the kept positions, 0 elsewhere)^T,
  * with the arithmetic of w4a16_gemm (exact products, FP32 sums, group scale in
  * FP32, BF16 RNE out) and its streaming kernel on 24% fewer weight bytes.
- * Shape rules for both: N % 16 == 0, K % 128 == 0; pointers 16-byte aligned.
+ * Shape rules for both: N % 32 == 0, K % 128 == 0; pointers 16-byte aligned.
  * ------------------------------------------------------------------------ */
 nvq_status int4_pack_sparse24(const void* w_bf16, const uint8_t* codes, const void* scales_bf16, int64_t N,
                               int64_t K, uint8_t* packed, void* packed_scales, void* stream);

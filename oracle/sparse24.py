@@ -18,9 +18,11 @@ the decode GEMM itself is the W4A16 one of ``oracle/int4.py``):
      i0 < i1 (0..3) as the nibble i0 | i1 << 2, and the two kept codes u.
   4. Y = X @ (s * (u - 8) at the kept positions, 0 elsewhere)^T in float64.
 
-Kernel order (``pack``): the 16-row tile x 128-k group "unit" of the decode
-kernel holds 512 bytes of codes, 256 bytes of metadata and 32 bytes of
-scales.  Inside a unit the m16n8k32 sparse MMA step s (0..3) reads the runs
+Kernel order (``pack``): the 32-row x 128-k group "unit" of the decode kernel
+is two 16-row tiles tt = 0, 1 (rows 16 tt .. 16 tt + 15), each 512 bytes of
+codes then 256 bytes of metadata (1536 bytes per unit), and 64 bytes of
+scales: 32-bit word 2 g + tt holds rows 16 tt + g (low half) and 16 tt + g + 8
+(high half).  Inside a tile the m16n8k32 sparse MMA step s (0..3) reads the runs
 G(s, j) = 8 s + j / 2 for even j and 8 s + 4 + (j - 1) / 2 for odd j (MMA
 run j = 0..7); lane (g, c) holds, for step s, one 32-bit word whose nibble
 i (bits 4i..4i+3) and nibble i + 4 are the two compressed values of its A
@@ -37,6 +39,7 @@ import numpy as np
 from . import int4 as oint4
 
 RUN = 4
+UNIT_ROWS = 32
 UNIT_CODE_BYTES = 512
 UNIT_META_BYTES = 256
 
@@ -96,80 +99,91 @@ def _mma_run(s: int, j: int) -> int:
     return 8 * s + (j // 2 if j % 2 == 0 else 4 + (j - 1) // 2)
 
 
+def _tile_words(kr: np.ndarray, meta: np.ndarray, r0: int, gi: int):
+    """Code words (32 lanes x 4 steps) and metadata words (16 lanes x 4 steps) of
+    the 16-row tile starting at row r0, group gi."""
+    codes = np.zeros(128, dtype=np.uint32)
+    metaw = np.zeros(64, dtype=np.uint32)
+    for lane in range(32):
+        g, c = lane >> 2, lane & 3
+        for s in range(4):
+            w = 0
+            for reg in range(4):
+                row = r0 + g + (8 if reg & 1 else 0)
+                kc = 2 * c + (8 if reg & 2 else 0)           # compressed k of the register's low half
+                for half_i, kk in enumerate((kc, kc + 1)):
+                    j, q = kk // 2, kk % 2
+                    run = 128 // RUN * gi + _mma_run(s, j)
+                    w |= int(kr[row, run, q]) << (4 * (reg + 4 * half_i))
+            codes[4 * lane + s] = w
+            if c < 2:
+                m = 0
+                for n in range(8):
+                    row = r0 + g + 8 * (n // 4)
+                    run = 128 // RUN * gi + _mma_run(s, 4 * c + n % 4)
+                    m |= int(meta[row, run]) << (4 * n)
+                metaw[4 * (2 * g + c) + s] = m
+    return codes, metaw
+
+
 def pack(u_kept: np.ndarray, meta: np.ndarray, s_bits: np.ndarray):
-    """Kernel order: (codes_and_meta uint8 [units * 768], scales uint8 [units * 32]),
-    units in (16-row tile, 128-k group) order, tile-major."""
+    """Kernel order: (codes_and_meta uint8 [units * 1536], scales uint8 [units * 64]),
+    units in (32-row tile, 128-k group) order, tile-major."""
     N, half = u_kept.shape
     K = 2 * half
-    assert N % 16 == 0 and K % 128 == 0
+    assert N % UNIT_ROWS == 0 and K % 128 == 0
     G = K // 128
     kr = u_kept.reshape(N, K // RUN, 2)
-    out = np.zeros((N // 16, G, UNIT_CODE_BYTES + UNIT_META_BYTES), dtype=np.uint8)
-    sc = np.zeros((N // 16, G, 32), dtype=np.uint8)
-    for nt in range(N // 16):
+    tb = UNIT_CODE_BYTES + UNIT_META_BYTES
+    out = np.zeros((N // UNIT_ROWS, G, 2, tb), dtype=np.uint8)
+    sc = np.zeros((N // UNIT_ROWS, G, 16, 2), dtype=np.uint16)
+    for nt in range(N // UNIT_ROWS):
         for gi in range(G):
-            codes = np.zeros(128, dtype=np.uint32)           # 32 lanes x 4 steps
-            metaw = np.zeros(64, dtype=np.uint32)            # 16 lanes (c = 0, 1) x 4 steps
-            for lane in range(32):
-                g, c = lane >> 2, lane & 3
-                for s in range(4):
-                    w = 0
-                    for reg in range(4):
-                        row = 16 * nt + g + (8 if reg & 1 else 0)
-                        kc = 2 * c + (8 if reg & 2 else 0)   # compressed k of the register's low half
-                        for half_i, kk in enumerate((kc, kc + 1)):
-                            j, q = kk // 2, kk % 2
-                            run = 128 // RUN * gi + _mma_run(s, j)
-                            val = int(kr[row, run, q])
-                            w |= val << (4 * (reg + 4 * half_i))
-                    codes[4 * lane + s] = w
-                    if c < 2:
-                        m = 0
-                        for n in range(8):
-                            row = 16 * nt + g + 8 * (n // 4)
-                            run = 128 // RUN * gi + _mma_run(s, 4 * c + n % 4)
-                            m |= int(meta[row, run]) << (4 * n)
-                        metaw[4 * (2 * g + c) + s] = m
-            out[nt, gi, :UNIT_CODE_BYTES] = codes.view(np.uint8)
-            out[nt, gi, UNIT_CODE_BYTES:] = metaw.view(np.uint8)
-            for g in range(8):
-                lo = s_bits[16 * nt + g, gi]
-                hi = s_bits[16 * nt + g + 8, gi]
-                sc[nt, gi, 4 * g:4 * g + 4] = np.array([lo & 0xFF, lo >> 8, hi & 0xFF, hi >> 8], dtype=np.uint8)
-    return out.reshape(-1), sc.reshape(-1)
+            for tt in range(2):
+                codes, metaw = _tile_words(kr, meta, UNIT_ROWS * nt + 16 * tt, gi)
+                out[nt, gi, tt, :UNIT_CODE_BYTES] = codes.view(np.uint8)
+                out[nt, gi, tt, UNIT_CODE_BYTES:] = metaw.view(np.uint8)
+                for g in range(8):
+                    sc[nt, gi, 2 * g + tt, 0] = s_bits[UNIT_ROWS * nt + 16 * tt + g, gi]
+                    sc[nt, gi, 2 * g + tt, 1] = s_bits[UNIT_ROWS * nt + 16 * tt + g + 8, gi]
+    return out.reshape(-1), sc.reshape(-1).view(np.uint8).copy()
 
 
 def unpack(packed: np.ndarray, packed_scales: np.ndarray, N: int, K: int):
     """Inverse of ``pack``: (u_kept, meta, s_bits)."""
     G = K // 128
-    p = np.asarray(packed, dtype=np.uint8).reshape(N // 16, G, UNIT_CODE_BYTES + UNIT_META_BYTES)
+    tb = UNIT_CODE_BYTES + UNIT_META_BYTES
+    p = np.asarray(packed, dtype=np.uint8).reshape(N // UNIT_ROWS, G, 2, tb)
     u = np.zeros((N, K // RUN, 2), dtype=np.uint8)
     meta = np.zeros((N, K // RUN), dtype=np.uint8)
-    for nt in range(N // 16):
+    for nt in range(N // UNIT_ROWS):
         for gi in range(G):
-            codes = p[nt, gi, :UNIT_CODE_BYTES].copy().view(np.uint32)
-            metaw = p[nt, gi, UNIT_CODE_BYTES:].copy().view(np.uint32)
-            for lane in range(32):
-                g, c = lane >> 2, lane & 3
-                for s in range(4):
-                    w = int(codes[4 * lane + s])
-                    for reg in range(4):
-                        row = 16 * nt + g + (8 if reg & 1 else 0)
-                        kc = 2 * c + (8 if reg & 2 else 0)
-                        for half_i, kk in enumerate((kc, kc + 1)):
-                            j, q = kk // 2, kk % 2
-                            run = 128 // RUN * gi + _mma_run(s, j)
-                            u[row, run, q] = (w >> (4 * (reg + 4 * half_i))) & 0xF
-                    if c < 2:
-                        m = int(metaw[4 * (2 * g + c) + s])
-                        for n in range(8):
-                            row = 16 * nt + g + 8 * (n // 4)
-                            run = 128 // RUN * gi + _mma_run(s, 4 * c + n % 4)
-                            meta[row, run] = (m >> (4 * n)) & 0xF
-    sc = np.asarray(packed_scales, dtype=np.uint8).reshape(N // 16, G, 32)
+            for tt in range(2):
+                r0 = UNIT_ROWS * nt + 16 * tt
+                codes = p[nt, gi, tt, :UNIT_CODE_BYTES].copy().view(np.uint32)
+                metaw = p[nt, gi, tt, UNIT_CODE_BYTES:].copy().view(np.uint32)
+                for lane in range(32):
+                    g, c = lane >> 2, lane & 3
+                    for s in range(4):
+                        w = int(codes[4 * lane + s])
+                        for reg in range(4):
+                            row = r0 + g + (8 if reg & 1 else 0)
+                            kc = 2 * c + (8 if reg & 2 else 0)
+                            for half_i, kk in enumerate((kc, kc + 1)):
+                                j, q = kk // 2, kk % 2
+                                run = 128 // RUN * gi + _mma_run(s, j)
+                                u[row, run, q] = (w >> (4 * (reg + 4 * half_i))) & 0xF
+                        if c < 2:
+                            m = int(metaw[4 * (2 * g + c) + s])
+                            for n in range(8):
+                                row = r0 + g + 8 * (n // 4)
+                                run = 128 // RUN * gi + _mma_run(s, 4 * c + n % 4)
+                                meta[row, run] = (m >> (4 * n)) & 0xF
+    sc = np.asarray(packed_scales, dtype=np.uint8).copy().view(np.uint16).reshape(N // UNIT_ROWS, G, 16, 2)
     s_bits = np.zeros((N, G), dtype=np.uint16)
-    for nt in range(N // 16):
-        for g in range(8):
-            s_bits[16 * nt + g] = sc[nt, :, 4 * g].astype(np.uint16) | (sc[nt, :, 4 * g + 1].astype(np.uint16) << 8)
-            s_bits[16 * nt + g + 8] = sc[nt, :, 4 * g + 2].astype(np.uint16) | (sc[nt, :, 4 * g + 3].astype(np.uint16) << 8)
+    for nt in range(N // UNIT_ROWS):
+        for w in range(16):
+            g, tt = w // 2, w % 2
+            s_bits[UNIT_ROWS * nt + 16 * tt + g] = sc[nt, :, w, 0]
+            s_bits[UNIT_ROWS * nt + 16 * tt + g + 8] = sc[nt, :, w, 1]
     return u.reshape(N, K // 2), meta, s_bits

@@ -104,10 +104,11 @@ namespace nvq {
 // 2:4 magnitude pruning of the BF16 master (two largest |w| of every run of four
 // k, the lower k on equal magnitudes) combined with the dense INT4 codes (a
 // run's largest |w| is always kept, so the group scales and the kept codes are
-// the dense ones), written in the sparse decode kernel's order: per 16-row x
-// 128-k unit, 512 bytes of A-fragment code words (lane-major, 4 m16n8k32 steps
-// per lane) and 256 bytes of metadata words (lanes c = 0, 1), then the unit's
-// 32 bytes of scales (word g: rows g (low half) and g + 8 (high half)).
+// the dense ones), written in the sparse decode kernel's order: per 32-row x
+// 128-k unit, two 16-row tiles tt, each 512 bytes of A-fragment code words
+// (lane-major, 4 m16n8k32 steps per lane) and 256 bytes of metadata words
+// (lanes c = 0, 1); the unit's 64 bytes of scales hold in word 2 g + tt rows
+// 16 tt + g (low half) and 16 tt + g + 8 (high half).
 
 // Kept positions (i0 < i1) of one run from its four bf16 values.
 __device__ __forceinline__ uint32_t run_meta(uint2 w4) {
@@ -129,18 +130,20 @@ __device__ __forceinline__ uint32_t sparse_run(uint32_t s, uint32_t j) {
   return 8 * s + ((j & 1u) ? 4 + (j >> 1) : (j >> 1));
 }
 
-// One thread per (unit, lane, step): one code word, and for lanes c < 2 one metadata word.
+// One thread per (unit, tile, lane, step): one code word, and for lanes c < 2 one metadata word.
 __global__ void int4_pack_sparse24_kernel(const uint2* __restrict__ w, const uint8_t* __restrict__ codes,
                                           const uint16_t* __restrict__ scales, uint32_t N, uint32_t K,
                                           uint32_t* __restrict__ packed, uint32_t* __restrict__ pscales) {
   const uint32_t G = K >> 7;
-  const uint64_t units = (uint64_t)(N >> 4) * G;
-  const uint64_t total = units * 128;
+  const uint64_t units = (uint64_t)(N >> 5) * G;
+  const uint64_t total = units * 256;
   for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (uint64_t)gridDim.x * blockDim.x) {
-    const uint64_t unit = i >> 7;
+    const uint64_t unit = i >> 8;
+    const uint32_t tt = (uint32_t)(i >> 7) & 1u;
     const uint32_t lane = (uint32_t)(i >> 2) & 31u, s = (uint32_t)i & 3u;
     const uint32_t g = lane >> 2, c = lane & 3u;
     const uint32_t nt = (uint32_t)(unit / G), gi = (uint32_t)(unit - (uint64_t)nt * G);
+    const uint32_t r0 = 32 * nt + 16 * tt;                  // first row of this 16-row tile
     auto kept_code = [&](uint32_t row, uint32_t run, uint32_t q) {   // q-th kept code of a run
       const uint32_t k0 = 128 * gi + 4 * run;
       const uint32_t m = run_meta(__ldg(w + ((size_t)row * K + k0) / 4));
@@ -150,7 +153,7 @@ __global__ void int4_pack_sparse24_kernel(const uint2* __restrict__ w, const uin
     uint32_t word = 0;
 #pragma unroll
     for (int reg = 0; reg < 4; ++reg) {
-      const uint32_t row = 16 * nt + g + ((reg & 1) ? 8u : 0u);
+      const uint32_t row = r0 + g + ((reg & 1) ? 8u : 0u);
       const uint32_t kc = 2 * c + ((reg & 2) ? 8u : 0u);   // compressed k of the register's low half
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -158,22 +161,22 @@ __global__ void int4_pack_sparse24_kernel(const uint2* __restrict__ w, const uin
         word |= kept_code(row, sparse_run(s, kk >> 1), kk & 1u) << (4 * (reg + 4 * h));
       }
     }
-    uint32_t* u = packed + unit * 192;                       // 768 bytes per unit
+    uint32_t* u = packed + unit * 384 + tt * 192;            // 1536 bytes per unit, 768 per tile
     u[4 * lane + s] = word;
     if (c < 2) {
       uint32_t m = 0;
 #pragma unroll
       for (int n = 0; n < 8; ++n) {
-        const uint32_t row = 16 * nt + g + 8 * (n >> 2);
+        const uint32_t row = r0 + g + 8 * (n >> 2);
         const uint32_t run = sparse_run(s, 4 * c + (n & 3));
         m |= run_meta(__ldg(w + ((size_t)row * K + 128 * gi + 4 * run) / 4)) << (4 * n);
       }
       u[128 + 4 * (2 * g + c) + s] = m;
     }
-    if (lane < 8 && s == 0) {                                // word g: rows g (low) and g + 8 (high)
-      const uint32_t lo = __ldg(scales + (size_t)(16 * nt + lane) * G + gi);
-      const uint32_t hi = __ldg(scales + (size_t)(16 * nt + lane + 8) * G + gi);
-      pscales[unit * 8 + lane] = lo | (hi << 16);
+    if (lane < 8 && s == 0) {                                // word 2 g + tt: rows r0 + g (low), + 8 (high)
+      const uint32_t lo = __ldg(scales + (size_t)(r0 + lane) * G + gi);
+      const uint32_t hi = __ldg(scales + (size_t)(r0 + lane + 8) * G + gi);
+      pscales[unit * 16 + 2 * lane + tt] = lo | (hi << 16);
     }
   }
 }

@@ -490,14 +490,14 @@ nvq_status int4_pack_sparse24(const void* w_bf16, const uint8_t* codes, const vo
                               int64_t K, uint8_t* packed, void* packed_scales, void* stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (N < 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "int4_pack_sparse24: bad sizes");
-  if (N % 16 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_pack_sparse24: need N % 16 == 0, K % 128 == 0");
+  if (N % 32 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_pack_sparse24: need N % 32 == 0, K % 128 == 0");
   if (N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "int4_pack_sparse24: too large");
   if (N == 0) return NVQ_OK;
   if (!w_bf16 || !codes || !scales_bf16 || !packed || !packed_scales)
     return fail(NVQ_ERR_INVALID_ARG, "int4_pack_sparse24: NULL pointer");
   if (!aligned16(w_bf16) || !aligned16(codes) || !aligned16(scales_bf16) || !aligned16(packed) || !aligned16(packed_scales))
     return fail(NVQ_ERR_MISALIGNED, "int4_pack_sparse24: pointer not 16-byte aligned");
-  const uint64_t threads = (uint64_t)(N / 16) * (uint64_t)(K / 128) * 128;
+  const uint64_t threads = (uint64_t)(N / 32) * (uint64_t)(K / 128) * 256;
   const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>((threads + 255) / 256, (uint64_t)sm_count() * 16));
   nvq::int4_pack_sparse24_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint2*>(w_bf16), codes,
                                                            static_cast<const uint16_t*>(scales_bf16), (uint32_t)N,
@@ -510,8 +510,8 @@ nvq_status w4a16_sparse24_gemm(const void* x_bf16, const uint8_t* packed, const 
                                int64_t M, int64_t N, int64_t K, void* stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "w4a16_sparse24_gemm: bad sizes");
-  if (N % 16 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_sparse24_gemm: need N % 16 == 0, K % 128 == 0");
-  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || (N / 16) * (K / 128) >= ((int64_t)1 << 32))
+  if (N % 32 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_sparse24_gemm: need N % 32 == 0, K % 128 == 0");
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || (N / 32) * (K / 128) >= ((int64_t)1 << 32))
     return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_sparse24_gemm: too large");
   if (M == 0) return NVQ_OK;
   if (!x_bf16 || !packed || !packed_scales || !y_bf16) return fail(NVQ_ERR_INVALID_ARG, "w4a16_sparse24_gemm: NULL pointer");

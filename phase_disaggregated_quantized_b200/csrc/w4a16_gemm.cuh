@@ -6,9 +6,9 @@
 // sharing one output tile by splitting K, partial sums added on chip).
 //
 // Work split.  The packed weights are a sequence of "units": one 128-wide
-// k-group of a tile of weight rows, tile-major.  Dense units hold 32 rows (two
-// 16-row MMA tiles: 2 KB of codes + 64 B of scales); 2:4-sparse units hold 16
-// rows (768 B of codes and metadata + 32 B of scales).  Each cluster of CS CTAs
+// k-group of a tile of weight rows, tile-major.  Units hold 32 rows (two 16-row
+// MMA tiles): dense 2 KB of codes + 64 B of scales, 2:4-sparse 1536 B of codes
+// and metadata + 64 B of scales.  Each cluster of CS CTAs
 // owns a contiguous run of whole tiles; inside the cluster the run's units are
 // split evenly over CS CTAs x W warps, so every warp streams the same number of
 // bytes whatever N and K are.
@@ -47,9 +47,10 @@ constexpr int CS = 2;                        // CTAs per cluster (74 such pairs 
 
 template <bool SPARSE>
 struct Unit {
-  static constexpr uint32_t TILES = SPARSE ? 1u : 2u;     // 16-row MMA tiles per unit
+  static constexpr uint32_t TILES = 2u;                   // 16-row MMA tiles per unit
   static constexpr uint32_t ROWS = 16u * TILES;           // weight rows of one output tile
-  static constexpr uint32_t CODE = SPARSE ? 768u : 2048u;
+  static constexpr uint32_t TILE_CODE = SPARSE ? 768u : 1024u;
+  static constexpr uint32_t CODE = TILES * TILE_CODE;
   static constexpr uint32_t SCALE = 32u * TILES;
   static constexpr uint32_t BYTES = CODE + SCALE;
 };
@@ -58,9 +59,10 @@ template <int NT8, bool SPARSE = false>
 struct Cfg {
   using U = Unit<SPARSE>;
   static constexpr int W = 8;                          // warps per CTA (two CTAs per SM)
-  static constexpr int SG = SPARSE ? 4 : 2;            // units per ring stage
+  static constexpr int SG = 2;                         // units per ring stage
   static constexpr int D = NT8 == 1 ? 3 : 6;           // ring stages per warp
   static constexpr int THREADS = W * 32;
+  static constexpr int MIN_CTAS = NT8 == 1 ? 2 : 1;     // CTAs per SM the register budget must allow
   static constexpr int STAGE = SG * U::BYTES;           // codes first, then the scales
   static constexpr int RING = W * D * STAGE;
   static constexpr int NTT = (int)U::TILES * NT8;       // 16 x 8 accumulator fragments per lane
@@ -314,33 +316,33 @@ __device__ __forceinline__ void mma_sp_acc(float (&d)[4], const uint32_t (&a)[4]
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3]), "r"(e));
 }
 
-// One 2:4-sparse unit (16 rows x 128 k, 64 kept codes per row): four m16n8k32
-// steps; step s reads runs 8 s .. 8 s + 7 of the group, so lane (g, c) needs
-// activations k = 32 s + 16 (c / 2) + {0 .. 15}, of which words c % 2, 2 + c % 2,
-// 4 + c % 2, 6 + c % 2 feed its B fragment.  d[t] receives the group sum.
+// One 2:4-sparse unit: two 16-row tiles x 128 k (64 kept codes per row), each
+// 512 bytes of code words and 256 of metadata words; four m16n8k32 steps per
+// tile.  Step s reads runs 8 s .. 8 s + 7 of the group, so lane (g, c) needs
+// activations k = 32 s + 16 (c / 2) + {0 .. 15}, of which words c % 2,
+// 2 + c % 2, 4 + c % 2, 6 + c % 2 feed its B fragment; the activations of a
+// step are loaded once for both tiles.  d[tt * NT8 + t] receives the group sum.
 template <int NT8, bool ONES>
-__device__ __forceinline__ void sparse_group(uint32_t unit, uint32_t lane, const uint4* const (&xrow)[NT8],
-                                             const bool (&live)[NT8], uint32_t gk, float (&d)[NT8][4]) {
+__device__ __forceinline__ void sparse_unit(uint32_t unit, uint32_t lane, const uint4* const (&xrow)[NT8],
+                                            const bool (&live)[NT8], uint32_t gk, float (&d)[2 * NT8][4]) {
   const uint32_t g = lane >> 2, c = lane & 3u, odd = c & 1u;
-  const uint4 wq = lds128(unit + lane * 16);
-  const uint4 mq = lds128(unit + 512 + (2 * g + odd) * 16);   // lanes c >= 2 load a copy the MMA ignores
-  const uint32_t wsw[4] = {wq.x, wq.y, wq.z, wq.w};
-  const uint32_t msw[4] = {mq.x, mq.y, mq.z, mq.w};
+  uint32_t wsw[2][4], msw[2][4];
+#pragma unroll
+  for (int tt = 0; tt < 2; ++tt) {
+    const uint4 wq = lds128(unit + tt * 768u + lane * 16);
+    const uint4 mq = lds128(unit + tt * 768u + 512 + (2 * g + odd) * 16);   // lanes c >= 2: a copy the MMA ignores
+    wsw[tt][0] = wq.x; wsw[tt][1] = wq.y; wsw[tt][2] = wq.z; wsw[tt][3] = wq.w;
+    msw[tt][0] = mq.x; msw[tt][1] = mq.y; msw[tt][2] = mq.z; msw[tt][3] = mq.w;
+  }
   constexpr uint32_t kNeg136 = 0xC308C308u;
   const uint32_t neg[4] = {kNeg136, kNeg136, kNeg136, kNeg136};
-  float t0[NT8][4], t1[NT8][4];
 #pragma unroll
-  for (int t = 0; t < NT8; ++t)
+  for (int t = 0; t < 2 * NT8; ++t)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) t0[t][e] = t1[t][e] = 0.f;
+    for (int e = 0; e < 4; ++e) d[t][e] = 0.f;
 #pragma unroll
   for (int st = 0; st < 4; ++st) {
-    uint32_t a[4];
-    word_to_frag(wsw[st], a);
-    if (!ONES) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = bf16x2_sub136(a[i]);
-    }
+    uint32_t b[NT8][4];
 #pragma unroll
     for (int t = 0; t < NT8; ++t) {
       uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
@@ -349,20 +351,30 @@ __device__ __forceinline__ void sparse_group(uint32_t unit, uint32_t lane, const
         x0 = __ldg(px);
         x1 = __ldg(px + 1);
       }
-      const uint32_t b[4] = {odd ? x0.y : x0.x, odd ? x0.w : x0.z, odd ? x1.y : x1.x, odd ? x1.w : x1.z};
-      float (&dd)[4] = (st & 1) ? t1[t] : t0[t];
-      mma_sp_acc(dd, a, b, msw[st]);
-      if (ONES) mma_sp_acc(dd, neg, b, msw[st]);
+      b[t][0] = odd ? x0.y : x0.x;
+      b[t][1] = odd ? x0.w : x0.z;
+      b[t][2] = odd ? x1.y : x1.x;
+      b[t][3] = odd ? x1.w : x1.z;
+    }
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      uint32_t a[4];
+      word_to_frag(wsw[tt][st], a);
+      if (!ONES) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = bf16x2_sub136(a[i]);
+      }
+#pragma unroll
+      for (int t = 0; t < NT8; ++t) {
+        mma_sp_acc(d[tt * NT8 + t], a, b[t], msw[tt][st]);
+        if (ONES) mma_sp_acc(d[tt * NT8 + t], neg, b[t], msw[tt][st]);
+      }
     }
   }
-#pragma unroll
-  for (int t = 0; t < NT8; ++t)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) d[t][e] = t0[t][e] + t1[t][e];
 }
 
 template <int NT8, bool SPARSE>
-__global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, 1) w4a16_kernel(
+__global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::MIN_CTAS) w4a16_kernel(
     const __nv_bfloat16* __restrict__ x, const uint8_t* __restrict__ pcodes, const uint8_t* __restrict__ pscales,
     __nv_bfloat16* __restrict__ y, uint32_t M, uint32_t N, uint32_t K) {
   using C = Cfg<NT8, SPARSE>;
@@ -486,7 +498,7 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, 1) w4a16_kernel(
           if ((uint32_t)i < n) {
             float d[NTT][4];
             if constexpr (SPARSE) {
-              sparse_group<NT8, C::ONES>(stage + i * UC, lane, xrow, live, g + i, d);
+              sparse_unit<NT8, C::ONES>(stage + i * UC, lane, xrow, live, g + i, d);
             } else if constexpr (C::XDB) {
               uint4 (&cur)[NT8][4] = (i & 1) ? xb : xa;
               uint4 (&nxt)[NT8][4] = (i & 1) ? xa : xb;

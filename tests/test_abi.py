@@ -175,12 +175,14 @@ def test_swiglu_gemm_host_rules(L):
 
 def test_sparse24_host_rules(L):
     p = L.int4_pack_sparse24
-    assert p(_vp(FAKE), _vp(FAKE), _vp(FAKE), 24, 128, _vp(FAKE), _vp(FAKE), None) == 2      # N % 16
+    assert p(_vp(FAKE), _vp(FAKE), _vp(FAKE), 24, 128, _vp(FAKE), _vp(FAKE), None) == 2      # N % 32
+    assert p(_vp(FAKE), _vp(FAKE), _vp(FAKE), 48, 128, _vp(FAKE), _vp(FAKE), None) == 2
     assert p(_vp(FAKE), _vp(FAKE), _vp(FAKE), 32, 100, _vp(FAKE), _vp(FAKE), None) == 2      # K % 128
     assert p(_vp(FAKE), None, _vp(FAKE), 32, 128, _vp(FAKE), _vp(FAKE), None) == 1
     assert p(_vp(FAKE), _vp(FAKE), _vp(FAKE), 32, 128, _vp(ODD), _vp(FAKE), None) == 3
     g = L.w4a16_sparse24_gemm
     assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 24, 128, None) == 2
+    assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 48, 128, None) == 2
     assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(ODD), 4, 256, 4096, None) == 3
     assert g(_vp(FAKE), None, _vp(FAKE), _vp(FAKE), 4, 256, 4096, None) == 1
     assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 0, 256, 4096, None) == 0

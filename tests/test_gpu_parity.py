@@ -349,7 +349,7 @@ def gpu_sparse24(w_cpu):
     return p, ps
 
 
-@pytest.mark.parametrize("N,K", [(16, 128), (64, 512), (48, 384)])
+@pytest.mark.parametrize("N,K", [(32, 128), (64, 512), (96, 384)])
 def test_sparse24_pack_bit_exact(N, K):
     from oracle import sparse24 as osp
     w = synth.weights(N, K, seed=N * 7 + K)
@@ -362,8 +362,8 @@ def test_sparse24_pack_bit_exact(N, K):
     np.testing.assert_array_equal(u8(ps), ops)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (4, 512, 1024), (8, 1024, 256), (13, 272, 384), (16, 512, 512),
-                                   (32, 1024, 2048), (40, 256, 1024), (1, 16, 128)])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (4, 512, 1024), (8, 1024, 256), (13, 288, 384), (16, 512, 512),
+                                   (32, 1024, 2048), (40, 256, 1024), (1, 32, 128)])
 def test_sparse24_decode_matches_oracle(M, N, K):
     from oracle import sparse24 as osp
     x = synth.activations(M, K, seed=M + 3 * K)

@@ -463,7 +463,7 @@ def test_sparse_pack_is_a_bijection_and_matches_hand_slots():
     meta = pairs[g.integers(0, 6, size=(N, K // 4))]
     s = g.integers(0, 1 << 16, size=(N, K // 128)).astype(np.uint16)
     p, ps = sparse24.pack(u, meta, s)
-    assert p.size == (N // 16) * (K // 128) * 768 and ps.size == (N // 16) * (K // 128) * 32
+    assert p.size == (N // 32) * (K // 128) * 1536 and ps.size == (N // 32) * (K // 128) * 64
     u2, m2, s2 = sparse24.unpack(p, ps, N, K)
     np.testing.assert_array_equal(u2, u)
     np.testing.assert_array_equal(m2, meta)
@@ -481,6 +481,11 @@ def test_sparse_pack_is_a_bijection_and_matches_hand_slots():
     assert (m0 & 0xF) == meta[0, 0] and ((m0 >> 4) & 0xF) == meta[0, 4] and ((m0 >> 16) & 0xF) == meta[8, 0]
     m1 = int(m[4 * 1 + 2])                                        # lane (0, 1), step 2: MMA runs 4..7
     assert (m1 & 0xF) == meta[0, 16 + 2] and ((m1 >> 4) & 0xF) == meta[0, 16 + 6]
+    t1 = p[768:768 + 512].copy().view(np.uint32)                  # unit 0, tile 1 = rows 16..31
+    assert (int(t1[0]) & 0xF) == kr[16, 0, 0] and ((int(t1[0]) >> 4) & 0xF) == kr[24, 0, 0]
+    assert (int(p[1536:1536 + 512].copy().view(np.uint32)[0]) & 0xF) == kr[0, 32, 0]   # unit 1: group 1
+    sw = ps.view("<u2")                                           # word 2g + tt: rows 16tt + g, + 8
+    assert sw[0] == s[0, 0] and sw[1] == s[8, 0] and sw[2] == s[16, 0] and sw[3] == s[24, 0] and sw[32] == s[0, 1]
 
 
 def test_sparse_w4a16_reference_against_explicit_loops():
