@@ -62,6 +62,17 @@ const char* nvq_last_error_detail(void);
  * a bounded wait, NVQ_ERR_CUDA if the synchronisation failed, else NVQ_OK. */
 nvq_status nvq_check_device_error(void* stream);
 
+/* Diagnostic of the timeout path: launches one thread on `stream` that waits,
+ * with the bounded wait every pipeline of this library uses, on an mbarrier
+ * that nothing ever completes.  After limit_ns of device time (1 us .. 100 ms,
+ * else NVQ_ERR_INVALID_ARG and nothing is launched) the wait gives up, raises
+ * the device error word and the kernel returns normally: no trap, no hang, the
+ * context stays usable.  The next nvq_check_device_error() then returns
+ * NVQ_ERR_DEVICE_TIMEOUT and clears the word.  Run it only while no other
+ * kernel of this library is in flight: a kernel that is waiting while the word
+ * is raised gives up too. */
+nvq_status nvq_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
 /* ------------------------------------------------------------------------ *
  * NVFP4 round-to-nearest quantization (Mix-Quant page, section 2: 16-element
  * groups with a local scale plus a tensor-level scale, plain RTN).

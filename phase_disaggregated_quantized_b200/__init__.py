@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
             "nvq_status_string": ([i32], ctypes.c_char_p),
             "nvq_last_error_detail": ([], ctypes.c_char_p),
             "nvq_check_device_error": ([vp], i32),
+            "nvq_selftest_wait_timeout": ([ctypes.c_uint64, vp], i32),
             "nvfp4_scales_bytes": ([i64, i64], sz),
             "nvfp4_quantize_workspace_bytes": ([i64, i64], sz),
             "nvfp4_quantize": ([vp, i64, i64, vp, vp, vp, vp, vp, sz, vp], i32),
@@ -125,6 +126,11 @@ def w4a16_workspace_bytes(M: int, N: int, K: int) -> int:
 
 def check_device_error(stream=None):
     _check(lib().nvq_check_device_error(_stream(stream)), "nvq_check_device_error")
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None):
+    """Launch the library's timeout diagnostic (one bounded wait that runs out)."""
+    _check(lib().nvq_selftest_wait_timeout(limit_ns, _stream(stream)), "nvq_selftest_wait_timeout")
 
 
 def nvfp4_quantize(x, tensor_scale_in=None, *, codes=None, scales=None, tensor_scale_out=None, workspace=None,

@@ -17,6 +17,19 @@
 #include "ptx.cuh"
 #include "w4a16_gemm.cuh"
 
+namespace nvq {
+// Diagnostic kernel: lane 0 initialises an mbarrier for one arrival that never
+// comes and waits for its first phase with the given limit.
+__global__ void bounded_wait_probe_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_addr(&bar);
+  mbar_init(b, 1);
+  fence_mbar_init();
+  mbar_wait_for(b, 0, limit_ns);
+}
+}  // namespace nvq
+
 namespace {
 
 thread_local char g_detail[256] = "";
@@ -216,6 +229,15 @@ nvq_status nvq_check_device_error(void* stream) {
     return fail(NVQ_ERR_DEVICE_TIMEOUT, "a kernel gave up on a bounded wait");
   }
   return NVQ_OK;
+}
+
+// One thread waits on an mbarrier that nothing completes, with the same bounded
+// wait the pipelines use, so the wait runs out and raises the error word.
+nvq_status nvq_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000ull || limit_ns > 100000000ull)
+    return fail(NVQ_ERR_INVALID_ARG, "nvq_selftest_wait_timeout: limit_ns outside [1 us, 100 ms]");
+  nvq::bounded_wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return launch_status("bounded_wait_probe_kernel");
 }
 
 // ------------------------------------------------------------------ NVFP4 quantize

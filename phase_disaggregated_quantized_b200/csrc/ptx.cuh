@@ -55,16 +55,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // (and raises the device error word) if it did not within kWaitLimitNs, or if
 // another part of the kernel has already raised it.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 1023u) == 0u) {
       if (error_raised()) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) { flag_error(kErrTimeout); return false; }
+      if (globaltimer() - t0 > limit_ns) { flag_error(kErrTimeout); return false; }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // Wait used while shutting down after an error: ignores the error word and

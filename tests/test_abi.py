@@ -18,7 +18,8 @@ def L():
 def test_header_lists_the_entry_points():
     names = nvq.header_functions()
     for must in ("nvfp4_quantize", "nvfp4_gemm_w4a4", "int4_pack_weights", "w4a16_gemm", "int4_quantize",
-                 "nvq_check_device_error", "nvfp4_scales_bytes", "w4a16_workspace_bytes"):
+                 "nvq_check_device_error", "nvq_selftest_wait_timeout", "nvfp4_scales_bytes",
+                 "w4a16_workspace_bytes"):
         assert must in names
 
 
@@ -86,6 +87,12 @@ def test_int4_calls_reject_bad_arguments(L):
     assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 48, 128, None, 0, None) == 2     # N % 32
     assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(ODD), 4, 256, 4096, None, 0, None) == 3    # y misaligned
     assert w(_vp(FAKE), _vp(FAKE), None, _vp(FAKE), 4, 256, 4096, None, 0, None) == 1         # NULL scales
+
+
+def test_timeout_selftest_rejects_limits_out_of_range(L):
+    assert L.nvq_selftest_wait_timeout(999, None) == 1              # below 1 us: nothing launched
+    assert L.nvq_selftest_wait_timeout(100_000_001, None) == 1      # above 100 ms
+    assert b"limit_ns" in L.nvq_last_error_detail()
 
 
 def test_zero_sized_calls_are_noops(L):

@@ -524,3 +524,21 @@ def test_prefill_streamed_matches_resident_weights():
 
 def test_device_error_word_is_clear_after_normal_runs():
     nvq.check_device_error()
+
+
+def test_bounded_wait_timeout_is_reported_and_context_stays_usable():
+    """A wait that nothing completes gives up after its limit, raises the error
+    word and returns; the host reads NVQ_ERR_DEVICE_TIMEOUT once, and the
+    kernels that follow still match the oracle."""
+    nvq.check_device_error()                                  # start clean
+    nvq.selftest_wait_timeout(2_000_000)                      # 2 ms
+    with pytest.raises(nvq.NvqError) as e:
+        nvq.check_device_error()
+    assert e.value.status == 6                                # NVQ_ERR_DEVICE_TIMEOUT
+    nvq.check_device_error()                                  # the check cleared the word
+    x = synth.activations(4, 512, seed=11)
+    w = synth.weights(256, 512, seed=12)
+    y, y_ref = w4a16_case(x, w)
+    ok, worst = onv.within_tolerance(y, y_ref)
+    assert ok, worst
+    nvq.check_device_error()
