@@ -471,28 +471,52 @@ def per_batch_decode(torch, nvq, dec, dec_w, stream, dec_bytes, reps: int = 20):
 
 def measure_e2e(torch, nvq, pre, stream, steps: int):
     """Prefill pass through the public binding with pinned host inputs/outputs:
-    H2D of each layer's activations, quantize + GEMM, D2H of each layer's output."""
+    H2D of each layer's activations, quantize + GEMM, D2H of each layer's output.
+    The copies run on two copy streams, so the next layers' inputs go up and the
+    finished layers' outputs come down while a layer is quantized and multiplied
+    (both PCIe directions at once); events order every buffer's reuse, within a
+    step and across steps."""
     hx = [torch.empty(L["x"].shape, dtype=torch.bfloat16, pin_memory=True) for L in pre]
     hy = [torch.empty(L["y"].shape, dtype=torch.bfloat16, pin_memory=True) for L in pre]
     for h, L in zip(hx, pre):
         h.copy_(L["x"].cpu())
     dx = [torch.empty_like(L["x"]) for L in pre]
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    x_in = [torch.cuda.Event() for _ in pre]        # layer i's input is on the device
+    x_used = [torch.cuda.Event() for _ in pre]      # layer i's quantize has read it
+    y_done = [torch.cuda.Event() for _ in pre]      # layer i's GEMM has written y
+    y_out = [torch.cuda.Event() for _ in pre]       # layer i's y is on the host
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    def one():
-        for L, h, d, hyy in zip(pre, hx, dx, hy):
-            d.copy_(h, non_blocking=True)
+    def one(first: bool):
+        for i, (L, h, d, hyy) in enumerate(zip(pre, hx, dx, hy)):
+            with torch.cuda.stream(up):
+                if not first:
+                    up.wait_event(x_used[i])                 # the last step's quantize is done with d
+                d.copy_(h, non_blocking=True)
+                x_in[i].record(up)
+            stream.wait_event(x_in[i])
             nvq.nvfp4_quantize(d, None, codes=L["xc"], scales=L["xs"], tensor_scale_out=L["tx"],
                                workspace=L["ws"], stream=stream)
+            x_used[i].record(stream)
+            if not first:
+                stream.wait_event(y_out[i])                  # the last step's y has left the device
             nvq.nvfp4_gemm_w4a4((L["xc"], L["xs"], L["tx"]), L["wq"], PREFILL_M, L["N"], L["K"], y=L["y"],
                                 stream=stream)
-            hyy.copy_(L["y"], non_blocking=True)
+            y_done[i].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(y_done[i])
+                hyy.copy_(L["y"], non_blocking=True)
+                y_out[i].record(down)
 
-    one()
+    one(True)
     torch.cuda.synchronize()
     a.record(stream)
+    up.wait_event(a)
+    down.wait_event(a)
     for _ in range(steps):
-        one()
+        one(False)
+    stream.wait_event(y_out[-1])                             # the step's last copy, after all others
     b.record(stream)
     torch.cuda.synchronize()
     secs = a.elapsed_time(b) / 1e3 / steps

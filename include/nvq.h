@@ -26,6 +26,9 @@
  *     wait that ran out) set a library-wide device error word that
  *     nvq_check_device_error() reads and clears.  No kernel traps.
  *   - Pointers must be 16-byte aligned (NVQ_ERR_MISALIGNED otherwise).
+ *   - Size limits common to all calls (NVQ_ERR_UNSUPPORTED_SHAPE beyond them):
+ *     every dimension < 2^31; a quantize call holds < 2^31 16-element blocks
+ *     (rows * K / 16); a GEMM has < 2^31 128 x 128 output blocks.
  */
 #ifndef NVQ_H_
 #define NVQ_H_

@@ -30,7 +30,7 @@ namespace nvq {
 
 constexpr int kAmaxThreads = 512;
 constexpr int kAmaxMaxBlocks = 592;       // 4 per SM on 148 SMs
-constexpr int kQuantThreads = 1024;   // two CTAs per SM: the per-CTA tables are built 296 times, not 1184
+constexpr int kQuantThreads = 1024;   // one CTA per SM (64 registers): the per-CTA tables are built 148 times
 
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t x, uint32_t y) {   // inputs already >= 0
   uint32_t r;
@@ -179,7 +179,7 @@ __device__ __forceinline__ uint32_t codes8_exact(const uint32_t* w, const uint32
 }
 
 // rows x K bf16 -> codes [rows, K/2], tiled scales, t.
-__global__ void __launch_bounds__(kQuantThreads, 2) nvfp4_quantize_kernel(
+__global__ void __launch_bounds__(kQuantThreads, 1) nvfp4_quantize_kernel(
     const uint4* __restrict__ x, uint32_t rows, uint32_t K, const float* __restrict__ t_in,
     const float* __restrict__ partial, int npartial, uint2* __restrict__ codes,
     uint8_t* __restrict__ scales, float* __restrict__ t_out) {
@@ -252,14 +252,21 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nvfp4_quantize_kernel(
   const uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x;
   uint32_t row = b0 / nbk, kb = b0 - row * nbk;
   const uint32_t step_r = stride / nbk, step_kb = stride - step_r * nbk;
+  // The next block's 32 bytes are requested before this one is processed, so
+  // the HBM latency of a tensor larger than L2 overlaps the conversion work.
+  uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
+  {
+    const uint32_t b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < nblocks) { p0 = __ldg(x + 2 * (size_t)b); p1 = __ldg(x + 2 * (size_t)b + 1); }
+  }
   for (uint32_t base = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); base < nblocks; base += stride) {
     const uint32_t b = base + lane;
     const bool valid = b < nblocks;                          // nblocks % 4 == 0: groups of 4 agree
-    uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (valid) {
-      const uint4 v0 = __ldg(x + 2 * (size_t)b), v1 = __ldg(x + 2 * (size_t)b + 1);
-      w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-      w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+    uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    {
+      const uint32_t bn = b + stride;                        // < 2^31 + one grid: no wrap
+      if (bn < nblocks) { p0 = __ldg(x + 2 * (size_t)bn); p1 = __ldg(x + 2 * (size_t)bn + 1); }
+      else { p0 = make_uint4(0, 0, 0, 0); p1 = p0; }
     }
     uint32_t a[8];
 #pragma unroll

@@ -92,6 +92,11 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uin
 }
 
 constexpr int64_t kMaxDim = (int64_t)1 << 31;
+// 16-element blocks of one quantize call, and output tiles of one GEMM: the
+// kernels step through them with 32-bit grid-stride counters, which stay below
+// 2^31 + one grid and so never wrap.
+constexpr int64_t kMaxBlocks = (int64_t)1 << 31;
+bool gemm_tiles_fit(int64_t M, int64_t N) { return ((M + 127) / 128) * ((N + 127) / 128) < kMaxBlocks; }
 
 // Decode launch: a persistent grid of clusters of nvq::w4a16::CS CTAs, as many
 // as can be resident at once (one CTA per SM), never more clusters than output
@@ -266,7 +271,7 @@ nvq_status quantize_validate(const char* name, const void* x_bf16, int64_t rows,
     snprintf(msg, sizeof(msg), "%s: K %% 64 != 0", name);
     return fail(NVQ_ERR_UNSUPPORTED_SHAPE, msg);
   }
-  if (rows >= kMaxDim || K >= kMaxDim || (rows * (K / 16)) >= ((int64_t)1 << 32)) {
+  if (rows >= kMaxDim || K >= kMaxDim || (rows * (K / 16)) >= kMaxBlocks) {
     snprintf(msg, sizeof(msg), "%s: tensor too large", name);
     return fail(NVQ_ERR_UNSUPPORTED_SHAPE, msg);
   }
@@ -298,7 +303,7 @@ nvq_status quantize_launch(const void* x_bf16, int64_t rows, int64_t K, const fl
   }
   const uint64_t nblocks = (uint64_t)rows * (uint64_t)(K / 16);
   const uint64_t want = (nblocks + nvq::kQuantThreads - 1) / nvq::kQuantThreads;
-  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count() * 2));
+  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count()));
   nvq::nvfp4_quantize_kernel<<<grid, nvq::kQuantThreads, 0, stream>>>(
       static_cast<const uint4*>(x_bf16), (uint32_t)rows, (uint32_t)K, tensor_scale_in, partial, amax_blocks,
       reinterpret_cast<uint2*>(codes), scales, tensor_scale_out);
@@ -315,7 +320,7 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const flo
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (rows < 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_quantize: rows < 0 or K <= 0");
   if (K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize: K % 64 != 0");
-  if (rows >= kMaxDim || K >= kMaxDim || (rows * (K / 16)) >= ((int64_t)1 << 32))
+  if (rows >= kMaxDim || K >= kMaxDim || (rows * (K / 16)) >= kMaxBlocks)
     return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize: tensor too large");
   if (tensor_scale_out == nullptr) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_quantize: tensor_scale_out is NULL");
   if (rows > 0 && (x_bf16 == nullptr || codes == nullptr || scales == nullptr))
@@ -340,7 +345,7 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const flo
   }
   const uint64_t nblocks = (uint64_t)rows * (uint64_t)(K / 16);
   const uint64_t want = (nblocks + nvq::kQuantThreads - 1) / nvq::kQuantThreads;
-  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count() * 2));
+  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count()));
   nvq::nvfp4_quantize_kernel<<<grid, nvq::kQuantThreads, 0, stream>>>(
       static_cast<const uint4*>(x_bf16), (uint32_t)rows, (uint32_t)K, tensor_scale_in,
       static_cast<const float*>(workspace), amax_blocks, reinterpret_cast<uint2*>(codes), scales,
@@ -410,7 +415,8 @@ nvq_status nvfp4_gemm_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, cons
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4: bad sizes");
   if (N % 8 != 0 || K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4: need N % 8 == 0, K % 64 == 0");
-  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4: too large");
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || !gemm_tiles_fit(M, N))
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4: too large");
   if (!x_codes || !x_scales || !t_x || !w_codes || !w_scales || !t_w || !y_bf16)
     return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4: NULL pointer");
   if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
@@ -429,7 +435,8 @@ nvq_status nvfp4_gemm_w4a4_swiglu(const uint8_t* x_codes, const uint8_t* x_scale
   if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4_swiglu: bad sizes");
   if (N % 256 != 0 || K % 64 != 0)
     return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4_swiglu: need N % 256 == 0, K % 64 == 0");
-  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4_swiglu: too large");
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim || !gemm_tiles_fit(M, N))
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_gemm_w4a4_swiglu: too large");
   if (!x_codes || !x_scales || !t_x || !w_codes || !w_scales || !t_w || !t_h || !h_codes || !h_scales)
     return fail(NVQ_ERR_INVALID_ARG, "nvfp4_gemm_w4a4_swiglu: NULL pointer");
   if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||

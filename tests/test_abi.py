@@ -64,6 +64,16 @@ def test_quantize_rejects_bad_arguments(L):
     assert b"workspace" in L.nvq_last_error_detail()
 
 
+def test_size_limits_keep_the_kernel_counters_from_wrapping(L):
+    # rows * K / 16 = 2^31 blocks: one past the limit of one quantize call
+    assert L.nvfp4_quantize(_vp(FAKE), 1 << 25, 1024, None, _vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE),
+                            1 << 20, None) == 2
+    assert L.nvfp4_quantize(_vp(FAKE), (1 << 25) - 1, 1024, None, _vp(FAKE), _vp(FAKE), _vp(FAKE), None,
+                            0, None) == 4     # just inside: reaches the workspace check
+    # (M / 128) * (N / 128) = 2^31 output blocks
+    assert L.nvfp4_gemm_w4a4(*([_vp(FAKE)] * 7), 1 << 24, 1 << 21, 64, None) == 2
+
+
 def test_gemm_rejects_bad_arguments(L):
     g = L.nvfp4_gemm_w4a4
     a = [_vp(FAKE)] * 7
