@@ -243,6 +243,11 @@ nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int6
  * after the wait).  So the packed weights must not be written by the kernel
  * immediately before it when that kernel lets dependents launch early; no
  * kernel of this library that writes them does, nor does an ordinary copy.
+ * It also lets the next kernel on the stream launch early (once its own wait
+ * is over, before it computes), so that kernel's CTAs fill the SMs this call
+ * frees: a kernel launched after it with programmatic dependent launch must
+ * execute griddepcontrol.wait before it reads y (ordinary launches are
+ * ordered as usual).
  * Shape rules: M >= 0, N % 32 == 0, K % 128 == 0.
  * ------------------------------------------------------------------------ */
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);

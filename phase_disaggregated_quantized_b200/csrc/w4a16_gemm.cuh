@@ -448,6 +448,10 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
   if (lane == 0)
     for (int s = 0; s < D && irem > 0; ++s) issue();
   grid_dependency_wait();                      // before any access to x or y
+  // Let the next kernel launch now: its CTAs take each SM slot that a CTA of
+  // this grid frees and request their own first weight stages during this
+  // grid's tail.  (Its own wait still holds its x and y until this grid is done.)
+  grid_launch_dependents();
 
   for (uint32_t pass = 0; pass < npass; ++pass) {
     const uint32_t m0 = pass * MC;
@@ -578,7 +582,6 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
       }
     }
 
-    if (pass + 1 == npass) grid_launch_dependents();   // the next kernel may start launching
     // ---- warps -> CTA: partial tiles summed in warp order through shared memory
     __syncthreads();                          // all rings idle: the slots may overlay them
     if (has0) put_tile<NTT>(wslots + (warp * 2 + 0) * TILEF + lane * 4 * NTT, p0);
