@@ -21,7 +21,7 @@ W4A4 NVFP4 path):
   4. Dequantized value = e2m1(code) * e4m3(s_b) * t, exact in float64.
   5. Y = Xhat @ What^T in float64.
 
-Readings where the pages are silent (each listed in the design doc): t = 1 for an
+Readings where the pages are silent: t = 1 for an
 all-zero tensor; t = amax/2688 in fp32; RNE for both roundings, saturating at
 448 and 6; zero codes under a zero scale; the sign of x kept on a zero code;
 the low nibble of a byte holds the even-k element.
