@@ -114,6 +114,30 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K,
                           void* stream);
 
 /* ------------------------------------------------------------------------ *
+ * One tensor's rows split over several processes (an M split of a prefill
+ * linear): the tensor-level scale of the Mix-Quant page, section 2, must come
+ * from the max |x| of the whole tensor, so each rank
+ *   1. nvfp4_amax            its rows' max |x| -> *amax_out (FP32, exact;
+ *                            0 for rows == 0);
+ *   2. all-reduces that FP32 value with MAX over the ranks (4 bytes);
+ *   3. nvfp4_scale_from_amax the combined value -> t, the same t that
+ *                            nvfp4_quantize computes for a tensor with that
+ *                            amax (1 if it is 0, else fp32_RNE(amax / 2688));
+ *   4. nvfp4_quantize        its rows with tensor_scale_in = that t.
+ * Every rank then holds exactly the codes and scales that one nvfp4_quantize
+ * call over the whole tensor would give for its rows (scales compared in the
+ * logical [rows, K/16] order; they tile identically when each shard starts on a
+ * multiple of 128 rows).
+ * nvfp4_amax: x_bf16, rows, K as for nvfp4_quantize; amax_out a 4-byte aligned
+ * device float; workspace of nvfp4_quantize_workspace_bytes(rows, K) bytes
+ * (may be NULL when rows == 0).  nvfp4_scale_from_amax: two 4-byte aligned
+ * device floats (may alias).  Both asynchronous on `stream`.
+ * ------------------------------------------------------------------------ */
+nvq_status nvfp4_amax(const void* x_bf16, int64_t rows, int64_t K, float* amax_out, void* workspace,
+                      size_t workspace_bytes, void* stream);
+nvq_status nvfp4_scale_from_amax(const float* amax, float* tensor_scale_out, void* stream);
+
+/* ------------------------------------------------------------------------ *
  * nvfp4_quantize without any device allocation or workspace (no counterpart
  * on the pages; an addition of this library).  For callers that cannot call
  * cudaMalloc or lend scratch memory: for example an engine whose device memory

@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
             "nvfp4_quantize_workspace_bytes": ([i64, i64], sz),
             "nvfp4_quantize": ([vp, i64, i64, vp, vp, vp, vp, vp, sz, vp], i32),
             "nvfp4_quantize_noalloc": ([vp, i64, i64, vp, vp, vp, vp, vp], i32),
+            "nvfp4_amax": ([vp, i64, i64, vp, vp, sz, vp], i32),
+            "nvfp4_scale_from_amax": ([vp, vp, vp], i32),
             "nvfp4_gemm_w4a4": ([vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
             "nvfp4_gemm_w4a4_swiglu": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
             "int4_quantize": ([vp, i64, i64, vp, vp, vp], i32),
@@ -154,6 +156,49 @@ def nvfp4_quantize(x, tensor_scale_in=None, *, codes=None, scales=None, tensor_s
                                 _ptr(tensor_scale_out), _ptr(workspace), ws_bytes, _stream(stream)),
            "nvfp4_quantize")
     return codes, scales, tensor_scale_out
+
+
+def nvfp4_amax(x, *, amax_out=None, workspace=None, stream=None):
+    """max |x| of a BF16 [rows, K] tensor -> float32 [1] on the device (0 for rows == 0)."""
+    _need_cuda(x, amax_out, workspace)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+    rows, K = x.shape
+    if amax_out is None:
+        amax_out = torch.empty(1, dtype=torch.float32, device=x.device)
+    need = nvfp4_quantize_workspace_bytes(rows, K)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().nvfp4_amax(_ptr(x), rows, K, _ptr(amax_out), _ptr(workspace), ws_bytes, _stream(stream)),
+           "nvfp4_amax")
+    return amax_out
+
+
+def nvfp4_scale_from_amax(amax, *, tensor_scale_out=None, stream=None):
+    """t of a tensor whose max |x| is amax (float32 [1] on the device) -> float32 [1]."""
+    _need_cuda(amax, tensor_scale_out)
+    if tensor_scale_out is None:
+        tensor_scale_out = torch.empty(1, dtype=torch.float32, device=amax.device)
+    _check(lib().nvfp4_scale_from_amax(_ptr(amax), _ptr(tensor_scale_out), _stream(stream)),
+           "nvfp4_scale_from_amax")
+    return tensor_scale_out
+
+
+def nvfp4_quantize_row_shard(x, group=None, *, codes=None, scales=None, stream=None):
+    """NVFP4-quantize this rank's rows of one tensor whose rows are split over
+    the ranks of a torch.distributed group, with the tensor scale of the whole
+    tensor: local max |x| (nvfp4_amax), a 4-byte all-reduce(MAX) over the group,
+    t from the result (nvfp4_scale_from_amax), then nvfp4_quantize with that t.
+    Returns (codes, scales, t) as nvfp4_quantize does."""
+    import torch.distributed as dist
+    amax = nvfp4_amax(x, stream=stream)
+    if stream is None:
+        dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
+    else:
+        with torch.cuda.stream(stream):
+            dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
+    t = nvfp4_scale_from_amax(amax, stream=stream)
+    return nvfp4_quantize(x, t, codes=codes, scales=scales, stream=stream)
 
 
 def nvfp4_quantize_noalloc(x, tensor_scale_in=None, *, codes, scales, tensor_scale_out, stream=None):

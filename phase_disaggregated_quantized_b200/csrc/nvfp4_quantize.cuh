@@ -72,6 +72,28 @@ __global__ void __launch_bounds__(kAmaxThreads) nvfp4_amax_kernel(const uint4* _
   }
 }
 
+// The tensor scale of a tensor whose max |x| is `amax`: 1 for an all-zero
+// tensor, else fp32_RNE(amax / 2688), 2688 = 6 (largest E2M1) x 448 (largest E4M3).
+__device__ __forceinline__ float tensor_scale_of(float amax) {
+  return amax == 0.f ? 1.0f : __fdiv_rn(amax, 2688.0f);
+}
+
+// Max of the amax kernel's per-CTA partials (0 for none): the tensor's max |x|.
+__global__ void __launch_bounds__(32) nvfp4_amax_finish_kernel(const float* __restrict__ partial, int npartial,
+                                                                float* __restrict__ amax_out) {
+  float m = 0.f;
+  for (int i = threadIdx.x; i < npartial; i += 32) m = fmaxf(m, __ldg(partial + i));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if (threadIdx.x == 0) *amax_out = m;
+}
+
+// t from a max |x| computed elsewhere (for instance combined over the row
+// shards of one tensor held by several processes).
+__global__ void nvfp4_scale_from_amax_kernel(const float* amax, float* t_out) {   // may alias
+  *t_out = tensor_scale_of(*amax);
+}
+
 // Value of a non-negative E4M3 (FN) code 0..126: bias 7, 3 mantissa bits.
 // Subnormals (exponent field 0) are m * 2^-9 = (1 + m/8) 2^-6 - 2^-6, exact.
 __device__ __forceinline__ float e4m3_value(uint32_t c) {
@@ -196,7 +218,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nvfp4_quantize_kernel(
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if (threadIdx.x == 0) {
-      const float t = t_in != nullptr ? __ldg(t_in) : (m == 0.f ? 1.0f : __fdiv_rn(m, 2688.0f));
+      const float t = t_in != nullptr ? __ldg(t_in) : tensor_scale_of(m);
       s_t = t;
       if (blockIdx.x == 0) *t_out = t;
     }

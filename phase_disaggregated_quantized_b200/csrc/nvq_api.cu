@@ -290,6 +290,14 @@ nvq_status quantize_validate(const char* name, const void* x_bf16, int64_t rows,
   return NVQ_OK;
 }
 
+// CTAs of the amax pre-pass over rows x K elements (rows > 0): four 16-byte
+// loads per thread per sweep, at most kAmaxMaxBlocks partials.
+int amax_grid(int64_t rows, int64_t K) {
+  const size_t nvec = (size_t)rows * (size_t)K / 8;
+  const size_t want = (nvec + 4 * nvq::kAmaxThreads - 1) / (4 * nvq::kAmaxThreads);
+  return (int)std::max<size_t>(1, std::min<size_t>(nvq::kAmaxMaxBlocks, want));
+}
+
 // amax pre-pass (when t is not given) into `partial[0 .. amax_blocks)`, then the quantize pass.
 nvq_status quantize_launch(const void* x_bf16, int64_t rows, int64_t K, const float* tensor_scale_in, uint8_t* codes,
                            uint8_t* scales, float* tensor_scale_out, float* partial, int amax_blocks,
@@ -331,9 +339,7 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const flo
   int amax_blocks = 0;
   if (need_amax) {
     const size_t nvec = (size_t)rows * (size_t)K / 8;
-    amax_blocks = (int)std::min<size_t>(nvq::kAmaxMaxBlocks, (nvec + 4 * nvq::kAmaxThreads - 1) /
-                                                                 (4 * nvq::kAmaxThreads));
-    if (amax_blocks < 1) amax_blocks = 1;
+    amax_blocks = amax_grid(rows, K);
     if (workspace == nullptr || workspace_bytes < (size_t)amax_blocks * sizeof(float))
       return fail(NVQ_ERR_WORKSPACE, "nvfp4_quantize: workspace missing or too small");
     if ((reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
@@ -351,6 +357,41 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const flo
       static_cast<const float*>(workspace), amax_blocks, reinterpret_cast<uint2*>(codes), scales,
       tensor_scale_out);
   return launch_status("nvfp4_quantize_kernel");
+}
+
+nvq_status nvfp4_amax(const void* x_bf16, int64_t rows, int64_t K, float* amax_out, void* workspace,
+                      size_t workspace_bytes, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (rows < 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_amax: rows < 0 or K <= 0");
+  if (K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_amax: K % 64 != 0");
+  if (rows >= kMaxDim || K >= kMaxDim || (rows * (K / 16)) >= kMaxBlocks)
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_amax: tensor too large");
+  if (amax_out == nullptr || (rows > 0 && x_bf16 == nullptr)) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_amax: NULL pointer");
+  if (!aligned16(x_bf16) || (reinterpret_cast<uintptr_t>(amax_out) & 3u) != 0)
+    return fail(NVQ_ERR_MISALIGNED, "nvfp4_amax: x not 16-byte or amax_out not 4-byte aligned");
+  int amax_blocks = 0;
+  if (rows > 0) {
+    amax_blocks = amax_grid(rows, K);
+    if (workspace == nullptr || workspace_bytes < (size_t)amax_blocks * sizeof(float))
+      return fail(NVQ_ERR_WORKSPACE, "nvfp4_amax: workspace missing or too small");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
+      return fail(NVQ_ERR_MISALIGNED, "nvfp4_amax: workspace not 4-byte aligned");
+    const size_t nvec = (size_t)rows * (size_t)K / 8;
+    nvq::nvfp4_amax_kernel<<<amax_blocks, nvq::kAmaxThreads, 0, stream>>>(static_cast<const uint4*>(x_bf16), nvec,
+                                                                           static_cast<float*>(workspace));
+    nvq_status st = launch_status("nvfp4_amax_kernel");
+    if (st != NVQ_OK) return st;
+  }
+  nvq::nvfp4_amax_finish_kernel<<<1, 32, 0, stream>>>(static_cast<const float*>(workspace), amax_blocks, amax_out);
+  return launch_status("nvfp4_amax_finish_kernel");
+}
+
+nvq_status nvfp4_scale_from_amax(const float* amax, float* tensor_scale_out, void* stream_) {
+  if (amax == nullptr || tensor_scale_out == nullptr) return fail(NVQ_ERR_INVALID_ARG, "nvfp4_scale_from_amax: NULL pointer");
+  if ((reinterpret_cast<uintptr_t>(amax) & 3u) != 0 || (reinterpret_cast<uintptr_t>(tensor_scale_out) & 3u) != 0)
+    return fail(NVQ_ERR_MISALIGNED, "nvfp4_scale_from_amax: pointer not 4-byte aligned");
+  nvq::nvfp4_scale_from_amax_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream_)>>>(amax, tensor_scale_out);
+  return launch_status("nvfp4_scale_from_amax_kernel");
 }
 
 // ------------------------------------------------------------------ NVFP4 GEMM

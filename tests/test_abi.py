@@ -19,6 +19,7 @@ def test_header_lists_the_entry_points():
     names = nvq.header_functions()
     for must in ("nvfp4_quantize", "nvfp4_gemm_w4a4", "int4_pack_weights", "w4a16_gemm", "int4_quantize",
                  "nvq_check_device_error", "nvq_selftest_wait_timeout", "nvfp4_scales_bytes",
+                 "nvfp4_amax", "nvfp4_scale_from_amax",
                  "w4a16_workspace_bytes"):
         assert must in names
 
@@ -97,6 +98,21 @@ def test_int4_calls_reject_bad_arguments(L):
     assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 48, 128, None, 0, None) == 2     # N % 32
     assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(ODD), 4, 256, 4096, None, 0, None) == 3    # y misaligned
     assert w(_vp(FAKE), _vp(FAKE), None, _vp(FAKE), 4, 256, 4096, None, 0, None) == 1         # NULL scales
+
+
+def test_row_shard_calls_reject_bad_arguments(L):
+    a = L.nvfp4_amax
+    assert a(_vp(FAKE), 4, 100, _vp(FAKE), _vp(FAKE), 1 << 20, None) == 2          # K % 64
+    assert a(_vp(FAKE), -1, 64, _vp(FAKE), _vp(FAKE), 1 << 20, None) == 1
+    assert a(_vp(FAKE), 4, 64, None, _vp(FAKE), 1 << 20, None) == 1                 # no amax_out
+    assert a(_vp(ODD), 4, 64, _vp(FAKE), _vp(FAKE), 1 << 20, None) == 3
+    assert a(_vp(FAKE), 4, 64, _vp(FAKE + 2), _vp(FAKE), 1 << 20, None) == 3        # amax_out not 4-aligned
+    assert a(_vp(FAKE), 4, 64, _vp(FAKE), None, 0, None) == 4                       # workspace
+    assert a(_vp(FAKE), 4, 64, _vp(FAKE), _vp(FAKE), 0, None) == 4
+    f = L.nvfp4_scale_from_amax
+    assert f(None, _vp(FAKE), None) == 1
+    assert f(_vp(FAKE), None, None) == 1
+    assert f(_vp(FAKE + 1), _vp(FAKE), None) == 3
 
 
 def test_timeout_selftest_rejects_limits_out_of_range(L):

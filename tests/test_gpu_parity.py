@@ -542,3 +542,37 @@ def test_bounded_wait_timeout_is_reported_and_context_stays_usable():
     ok, worst = onv.within_tolerance(y, y_ref)
     assert ok, worst
     nvq.check_device_error()
+
+
+@pytest.mark.parametrize("rows,K,cut", [(384, 512, 128), (256, 4096, 128), (300, 192, 256)])
+def test_row_split_quantize_matches_one_whole_tensor_call(rows, K, cut):
+    """Rows split into two shards at `cut`: per-shard nvfp4_amax, their max (the
+    all-reduce(MAX) across ranks, here on one device), nvfp4_scale_from_amax,
+    then nvfp4_quantize of each shard with that t give the bytes of one call
+    over the whole tensor, and the oracle's t."""
+    x = synth.activations(rows, K, seed=rows + K, n_outliers=3).cuda()
+    whole_c, whole_s, whole_t = nvq.nvfp4_quantize(x)
+    shards = [x[:cut].contiguous(), x[cut:].contiguous()]
+    amaxes = [nvq.nvfp4_amax(sh) for sh in shards]
+    amax = torch.maximum(amaxes[0], amaxes[1])
+    t = nvq.nvfp4_scale_from_amax(amax)
+    parts = [nvq.nvfp4_quantize(sh, t) for sh in shards]
+    nvq.check_device_error()
+    assert float(amax.item()) == float(bf16_to_f64(x.cpu()).__abs__().max())
+    assert float(t.item()) == onv.tensor_scale(bf16_to_f64(x.cpu())) == float(whole_t.item())
+    assert torch.equal(torch.cat([parts[0][0], parts[1][0]]), whole_c)
+    logical = [onv.scales_from_tiled(u8(p[1]), sh.shape[0], K) for p, sh in zip(parts, shards)]
+    np.testing.assert_array_equal(np.concatenate(logical), onv.scales_from_tiled(u8(whole_s), rows, K))
+
+
+def test_amax_of_empty_and_zero_shards_and_scale_of_zero():
+    z = torch.zeros(0, 128, dtype=torch.bfloat16, device="cuda")
+    assert float(nvq.nvfp4_amax(z).item()) == 0.0
+    zero = torch.zeros(64, 128, dtype=torch.bfloat16, device="cuda")
+    a = nvq.nvfp4_amax(zero)
+    assert float(a.item()) == 0.0
+    assert float(nvq.nvfp4_scale_from_amax(a).item()) == 1.0              # the all-zero reading
+    for v in (1.0, 2688.0, 3.0e-30, 1.0e30, 448.0 * 6.0 * 7.0):
+        t = nvq.nvfp4_scale_from_amax(torch.tensor([v], dtype=torch.float32, device="cuda"))
+        assert float(t.item()) == onv.tensor_scale_from_amax(float(np.float32(v)))
+    nvq.check_device_error()
