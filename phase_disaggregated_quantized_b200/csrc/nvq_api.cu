@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/nvq.h"
@@ -108,7 +109,7 @@ nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* 
                         cudaStream_t stream) {
   using C = nvq::w4a16::Cfg<NT8, SPARSE>;
   auto fn = nvq::w4a16::w4a16_kernel<NT8, SPARSE>;
-  static int max_clusters[kMaxDevices] = {};     // 0: not queried yet on that device
+  static std::atomic<int> max_clusters[kMaxDevices];   // 0: not queried yet on that device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm: cudaGetDevice");
@@ -126,18 +127,18 @@ nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* 
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (max_clusters[dev] == 0) {
+  int maxc = max_clusters[dev].load(std::memory_order_acquire);
+  if (maxc == 0) {                              // two threads may both get here: same result
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm: shared memory attribute");
     cfg.gridDim = dim3(nvq::w4a16::CS, 1, 1);
-    int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, fn, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&maxc, fn, &cfg);
     if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm: cudaOccupancyMaxActiveClusters");
-    if (n < 1) return fail(NVQ_ERR_CUDA, "w4a16_gemm: no cluster of the decode kernel fits on this GPU");
-    max_clusters[dev] = n;
+    if (maxc < 1) return fail(NVQ_ERR_CUDA, "w4a16_gemm: no cluster of the decode kernel fits on this GPU");
+    max_clusters[dev].store(maxc, std::memory_order_release);
   }
   const int64_t tiles = N / nvq::w4a16::Unit<SPARSE>::ROWS;
-  const int64_t nclu = std::min<int64_t>(max_clusters[dev], tiles);
+  const int64_t nclu = std::min<int64_t>(maxc, tiles);
   cfg.gridDim = dim3((unsigned)(nclu * nvq::w4a16::CS), 1, 1);
   cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, fn, static_cast<const __nv_bfloat16*>(x), pc, static_cast<const uint8_t*>(ps),
@@ -434,12 +435,18 @@ nvq_status launch_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const fl
   p.h_scales = h_scales;
   p.t_h = t_h;
   p.h_katoms = (uint32_t)(N / 2 / 64);
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(nvfp4_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  // The shared-memory opt-in is a per-device setting of the kernel: once per device.
+  int dev = 0;
+  const cudaError_t de = cudaGetDevice(&dev);
+  if (de != cudaSuccess) return cuda_fail(de, "nvfp4_gemm_w4a4: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(NVQ_ERR_CUDA, "nvfp4_gemm_w4a4: device index out of range");
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t attr_err[kMaxDevices];   // zero = cudaSuccess
+  std::call_once(once[dev], [dev] {
+    attr_err[dev] = cudaFuncSetAttribute(nvfp4_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_BYTES);
   });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "nvfp4_gemm_w4a4: smem attribute");
+  if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "nvfp4_gemm_w4a4: smem attribute");
   const uint64_t tiles = (uint64_t)p.num_m_tiles * p.num_n_tiles;
   const int grid = (int)std::min<uint64_t>(tiles, (uint64_t)sm_count());
   nvfp4_gemm_kernel<EPI><<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, my, p);
