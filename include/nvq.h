@@ -60,6 +60,19 @@ const char* nvq_status_string(nvq_status s);
  * error), or "" if none; owned by the library, valid until the next call. */
 const char* nvq_last_error_detail(void);
 
+/* Workspace bytes of one call, by operation (the per-operation *_workspace_bytes
+ * functions give the same numbers): NVQ_OP_NVFP4_QUANTIZE (rows = M, K; also
+ * nvfp4_amax), NVQ_OP_NVFP4_GEMM (0: none), NVQ_OP_W4A16_GEMM (0: partial sums
+ * stay on chip), NVQ_OP_LINEAR (nvq_linear at the default crossover).
+ * SIZE_MAX for an unknown op. */
+typedef enum {
+  NVQ_OP_NVFP4_QUANTIZE = 0,
+  NVQ_OP_NVFP4_GEMM = 1,
+  NVQ_OP_W4A16_GEMM = 2,
+  NVQ_OP_LINEAR = 3
+} nvq_op;
+size_t nvq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
+
 /* Synchronises `stream`, then reads and clears the device error word.
  * Returns NVQ_ERR_DEVICE_TIMEOUT if any kernel since the last check gave up on
  * a bounded wait, NVQ_ERR_CUDA if the synchronisation failed, else NVQ_OK. */
@@ -107,6 +120,12 @@ nvq_status nvq_selftest_wait_timeout(uint64_t limit_ns, void* stream);
  *                   bytes (may be NULL when that is 0).
  * ------------------------------------------------------------------------ */
 size_t nvfp4_scales_bytes(int64_t rows, int64_t K);
+/* Host-side map of the tiled scale layout: byte offset, inside the scales
+ * buffer of a [rows, K] tensor, of the E4M3 scale of row `row`, 16-element
+ * block `kblock`; -1 if an argument is out of range.  The layout is 512-byte
+ * atoms of 128 rows x 4 blocks, row-tile major, each atom the 32 x 16-byte
+ * matrix the block-scaled tensor-core MMA takes its scales from. */
+int64_t nvfp4_scale_offset(int64_t row, int64_t kblock, int64_t rows, int64_t K);
 size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K);
 nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K,
                           const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,

@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
             "nvq_check_device_error": ([vp], i32),
             "nvq_selftest_wait_timeout": ([ctypes.c_uint64, vp], i32),
             "nvfp4_scales_bytes": ([i64, i64], sz),
+            "nvfp4_scale_offset": ([i64, i64, i64, i64], i64),
+            "nvq_workspace_bytes": ([i32, i64, i64, i64], sz),
             "nvfp4_quantize_workspace_bytes": ([i64, i64], sz),
             "nvfp4_quantize": ([vp, i64, i64, vp, vp, vp, vp, vp, sz, vp], i32),
             "nvfp4_quantize_noalloc": ([vp, i64, i64, vp, vp, vp, vp, vp], i32),
@@ -116,6 +118,18 @@ def _need_cuda(*ts):
 
 def nvfp4_scales_bytes(rows: int, K: int) -> int:
     return int(lib().nvfp4_scales_bytes(rows, K))
+
+
+NVQ_OP_NVFP4_QUANTIZE, NVQ_OP_NVFP4_GEMM, NVQ_OP_W4A16_GEMM, NVQ_OP_LINEAR = 0, 1, 2, 3
+
+
+def nvfp4_scale_offset(row: int, kblock: int, rows: int, K: int) -> int:
+    """Byte offset of the scale of (row, 16-element block) in the tiled scales of a [rows, K] tensor (-1: out of range)."""
+    return int(lib().nvfp4_scale_offset(row, kblock, rows, K))
+
+
+def nvq_workspace_bytes(op: int, M: int, N: int, K: int) -> int:
+    return int(lib().nvq_workspace_bytes(op, M, N, K))
 
 
 def nvfp4_quantize_workspace_bytes(rows: int, K: int) -> int:

@@ -252,6 +252,16 @@ size_t nvfp4_scales_bytes(int64_t rows, int64_t K) {
   return (size_t)((rows + 127) / 128 * 128) * (size_t)(K / 16);
 }
 
+// 512-byte atoms of 128 rows x 4 blocks, row-tile major: the atom of (row, kb)
+// is (row / 128) * (K / 64) + kb / 4; inside it the byte is 16 (row % 32) +
+// 4 ((row % 128) / 32) + kb % 4 -- the 32 x 16-byte matrix whose column c holds
+// rows 32 c + lane, as the block-scaled MMA reads scales from TMEM.
+int64_t nvfp4_scale_offset(int64_t row, int64_t kblock, int64_t rows, int64_t K) {
+  if (rows <= 0 || K <= 0 || K % 64 != 0 || row < 0 || row >= rows || kblock < 0 || kblock >= K / 16) return -1;
+  const int64_t atom = (row / 128) * (K / 64) + kblock / 4;
+  return atom * 512 + 16 * (row % 32) + 4 * ((row % 128) / 32) + kblock % 4;
+}
+
 size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K) {
   if (rows <= 0 || K <= 0) return 0;
   return (size_t)nvq::kAmaxMaxBlocks * sizeof(float);
@@ -612,6 +622,16 @@ size_t nvq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t cross
   if (crossover_m < 0) crossover_m = kDefaultCrossoverM;
   if (M <= crossover_m || M <= 0 || K <= 0 || K % 64 != 0) return 0;
   return linear_ws_layout(M, K).total;
+}
+
+size_t nvq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
+  switch (op) {
+    case NVQ_OP_NVFP4_QUANTIZE: return nvfp4_quantize_workspace_bytes(M, K);
+    case NVQ_OP_NVFP4_GEMM: return 0;
+    case NVQ_OP_W4A16_GEMM: return w4a16_workspace_bytes(M, N, K);
+    case NVQ_OP_LINEAR: return nvq_linear_workspace_bytes(M, N, K, -1);
+  }
+  return SIZE_MAX;
 }
 
 nvq_status nvq_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, const uint8_t* w_codes,

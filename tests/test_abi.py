@@ -19,7 +19,7 @@ def test_header_lists_the_entry_points():
     names = nvq.header_functions()
     for must in ("nvfp4_quantize", "nvfp4_gemm_w4a4", "int4_pack_weights", "w4a16_gemm", "int4_quantize",
                  "nvq_check_device_error", "nvq_selftest_wait_timeout", "nvfp4_scales_bytes",
-                 "nvfp4_amax", "nvfp4_scale_from_amax",
+                 "nvfp4_amax", "nvfp4_scale_from_amax", "nvfp4_scale_offset", "nvq_workspace_bytes",
                  "w4a16_workspace_bytes"):
         assert must in names
 
@@ -44,6 +44,28 @@ def test_size_helpers(L):
     assert L.w4a16_workspace_bytes(1, 4096, 4096) == 0          # partial sums stay on chip
     assert L.w4a16_workspace_bytes(4, 256, 4096) == 0
     assert L.w4a16_workspace_bytes(4096, 4096, 4096) == 0
+
+
+def test_scale_offset_map_matches_the_oracles_layout(L):
+    import numpy as np
+    from oracle import nvfp4 as onv
+    for rows, K in ((1, 64), (130, 512), (300, 192), (256, 1024)):
+        want = onv.scale_offsets(rows, K)
+        got = np.array([[L.nvfp4_scale_offset(r, kb, rows, K) for kb in range(K // 16)] for r in range(rows)])
+        np.testing.assert_array_equal(got, want)
+        assert sorted(got.ravel().tolist()) == sorted(set(got.ravel().tolist()))     # one byte per scale
+        assert got.max() < L.nvfp4_scales_bytes(rows, K)
+    for bad in ((-1, 0, 4, 64), (4, 0, 4, 64), (0, 4, 4, 64), (0, -1, 4, 64), (0, 0, 4, 100), (0, 0, 0, 64)):
+        assert L.nvfp4_scale_offset(*bad) == -1
+
+
+def test_workspace_bytes_by_operation(L):
+    assert L.nvq_workspace_bytes(0, 8192, 0, 4096) == L.nvfp4_quantize_workspace_bytes(8192, 4096) > 0
+    assert L.nvq_workspace_bytes(1, 8192, 4096, 4096) == 0
+    assert L.nvq_workspace_bytes(2, 16, 4096, 4096) == L.w4a16_workspace_bytes(16, 4096, 4096) == 0
+    assert L.nvq_workspace_bytes(3, 4096, 24576, 4096) == L.nvq_linear_workspace_bytes(4096, 24576, 4096, -1) > 0
+    assert L.nvq_workspace_bytes(3, 1, 24576, 4096) == 0
+    assert L.nvq_workspace_bytes(7, 1, 1, 64) == 2 ** 64 - 1
 
 
 FAKE = 0x7F0000000000          # 16-byte aligned, never dereferenced: validation fails first
