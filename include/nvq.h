@@ -165,15 +165,19 @@ nvq_status nvfp4_scale_from_amax(const float* amax, float* tensor_scale_out, voi
  * as nvfp4_quantize, minus the workspace.
  *
  * The tensor-amax partials live in a fixed 4 KiB file-scope device array
- * inside the library (1024 floats, one partial per 2^20 input elements), held
- * on every GPU that loads the library until the process exits.  Limit:
- * rows * K <= 2^30 elements; larger calls return NVQ_ERR_UNSUPPORTED_SHAPE.
+ * inside the library (1024 floats; the amax pre-pass uses the same grid as
+ * nvfp4_quantize, at most 592 partials), held on every GPU that loads the
+ * library until the process exits.  Limit: rows * K <= 2^30 elements; larger
+ * calls return NVQ_ERR_UNSUPPORTED_SHAPE before any pointer is examined.
  * The first call on each device resolves the array's device address with
- * cudaGetSymbolAddress (that device must be current); make that first call
- * before any stream capture.  All calls on a device share the array: calls
- * that overlap on the GPU (different streams, no ordering) race and give wrong
- * results.  Each call overwrites every partial it later reads, so nothing
- * needs clearing between calls.  Calls no cudaMalloc/cudaFree.
+ * cudaGetSymbolAddress (that device must be current) and caches it for the
+ * life of the process; make that first call before any stream capture.  The
+ * cached address does not survive cudaDeviceReset() or a reset of the primary
+ * context: do not call this entry point after either.  All calls on a device
+ * share the array: calls that overlap on the GPU (different streams, no
+ * ordering) race and give wrong results.  Each call overwrites every partial
+ * it later reads, so nothing needs clearing between calls.  Calls no
+ * cudaMalloc/cudaFree.
  * ------------------------------------------------------------------------ */
 nvq_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t K,
                                   const float* tensor_scale_in, uint8_t* codes, uint8_t* scales,

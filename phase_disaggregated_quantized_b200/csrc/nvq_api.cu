@@ -740,8 +740,11 @@ nvq_status nvq_prefill_streamed(const nvq_stream_layer* layers, int n, int64_t M
 namespace {
 
 constexpr int kNoallocPartials = 1024;                   // scratch capacity (floats)
-constexpr int64_t kNoallocElemsPerPartial = (int64_t)1 << 20;
+constexpr int64_t kNoallocMaxElems = (int64_t)1 << 30;   // largest rows * K this entry point takes
 constexpr int kNoallocMaxDevices = 64;
+// The amax pre-pass uses the same grid as nvfp4_quantize, never more CTAs
+// (partials) than the array holds.
+static_assert(nvq::kAmaxMaxBlocks <= kNoallocPartials, "amax partials must fit the fixed scratch");
 
 static __device__ __align__(256) float g_noalloc_amax_partials[kNoallocPartials];
 
@@ -749,7 +752,7 @@ std::mutex g_noalloc_mutex;
 float* g_noalloc_scratch[kNoallocMaxDevices] = {};
 
 // Device address of the scratch array on the current device, resolved once per
-// device (with that device current) and cached.
+// device (with that device current) and cached for the life of the process.
 nvq_status noalloc_scratch(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -772,18 +775,21 @@ extern "C" {
 
 nvq_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t K, const float* tensor_scale_in,
                                   uint8_t* codes, uint8_t* scales, float* tensor_scale_out, void* stream_) {
+  // The size limit comes first: an oversized call is rejected before any
+  // pointer is looked at.
+  if (rows > 0 && K > 0 && rows > kNoallocMaxElems / K)
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE,
+                "nvfp4_quantize_noalloc: rows*K exceeds 2^30 elements, the largest tensor this entry point "
+                "takes; use nvfp4_quantize with a workspace");
   nvq_status st = quantize_validate("nvfp4_quantize_noalloc", x_bf16, rows, K, codes, scales, tensor_scale_out);
   if (st != NVQ_OK) return st;
-  if (rows * K > (int64_t)kNoallocPartials * kNoallocElemsPerPartial)
-    return fail(NVQ_ERR_UNSUPPORTED_SHAPE,
-                "nvfp4_quantize_noalloc: rows*K exceeds 2^30 elements (the fixed scratch holds 1024 partial maxima, "
-                "one per 2^20 elements); use nvfp4_quantize with a workspace");
+  int amax_blocks = 0;
+  if (tensor_scale_in == nullptr && rows > 0) amax_blocks = amax_grid(rows, K);
+  if (amax_blocks > kNoallocPartials)
+    return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize_noalloc: amax partials exceed the fixed scratch");
   float* scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != NVQ_OK) return st;
-  int amax_blocks = 0;
-  if (tensor_scale_in == nullptr && rows > 0)
-    amax_blocks = (int)((rows * K + kNoallocElemsPerPartial - 1) / kNoallocElemsPerPartial);
   return quantize_launch(x_bf16, rows, K, tensor_scale_in, codes, scales, tensor_scale_out, scratch, amax_blocks,
                          static_cast<cudaStream_t>(stream_));
 }
