@@ -44,13 +44,71 @@ def gate_up_ref(xhat: np.ndarray, wg_hat: np.ndarray, wu_hat: np.ndarray):
     return G, U, silu(G) * U
 
 
-def error_band(G: np.ndarray, U: np.ndarray) -> np.ndarray:
-    """|H' - H| allowed for an H' made from G', U' inside the GEMM bar
-    (|G' - G| <= 8e-3 |G| + 1e-3 rms(G), same for U), to first order:
-    |silu'(g)| |u| dG + |silu(g)| dU, with |silu'| <= 1.1."""
+def silu_prime(g: np.ndarray) -> np.ndarray:
+    """d/dg silu(g) = sigmoid(g) (1 + g (1 - sigmoid(g))), float64."""
+    g = np.asarray(g, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        sg = 1.0 / (1.0 + np.exp(-g))
+    return sg * (1.0 + g * (1.0 - sg))
+
+
+def _silu_second(g: float) -> float:
+    sg = 1.0 / (1.0 + np.exp(-g))
+    return sg * (1.0 - sg) * (2.0 + g * (1.0 - 2.0 * sg))
+
+
+def _bisect(f, a: float, b: float) -> float:
+    fa = f(a)
+    for _ in range(200):
+        m = 0.5 * (a + b)
+        fm = f(m)
+        if (fm > 0) == (fa > 0):
+            a, fa = m, fm
+        else:
+            b = m
+    return 0.5 * (a + b)
+
+
+# silu' has exactly two local extrema (the zeros of silu''): a minimum near
+# g = -2.3994 and a maximum near g = +2.3994; it tends to 0 and to 1 at -inf
+# and +inf.  So over an interval max |silu'| is attained at an end or at one of
+# these two points.
+SILU_PRIME_EXTREMA = (_bisect(_silu_second, -4.0, -1.0), _bisect(_silu_second, 1.0, 4.0))
+
+
+def max_abs_silu_prime(lo: np.ndarray, hi: np.ndarray) -> np.ndarray:
+    """max |silu'(g)| over g in [lo, hi] (elementwise, lo <= hi)."""
+    m = np.maximum(np.abs(silu_prime(lo)), np.abs(silu_prime(hi)))
+    for c in SILU_PRIME_EXTREMA:
+        inside = (lo <= c) & (c <= hi)
+        m = np.where(inside, np.maximum(m, abs(float(silu_prime(c)))), m)
+    return m
+
+
+def error_band(G: np.ndarray, U: np.ndarray, rel_eval: float = 0.0) -> np.ndarray:
+    """Largest |H' - H| for H' = silu(G') U' with G', U' inside the GEMM bar
+    (|G' - G| <= dG = 8e-3 |G| + 1e-3 rms(G), the same for U), H = silu(G) U.
+
+    silu(G') U' - silu(G) U = (silu(G') - silu(G)) U' + silu(G) (U' - U), and by
+    the mean value theorem |silu(G') - silu(G)| <= L dG with L the largest
+    |silu'| over [G - dG, G + dG]; |U'| <= |U| + dU.  Hence
+        band = L dG (|U| + dU) + |silu(G)| dU.
+    The bound is reached up to the variation of silu' over the interval (the
+    signs of G' - G and U' - U can be chosen to align both terms), so it is at
+    most about twice the true largest deviation.
+
+    rel_eval adds rel_eval * (|silu(G)| + L dG) (|U| + dU): a relative error of
+    the silu evaluation itself, for a comparison with an implementation that
+    evaluates silu approximately."""
+    G = np.asarray(G, dtype=np.float64)
+    U = np.asarray(U, dtype=np.float64)
     dG = 8e-3 * np.abs(G) + 1e-3 * float(np.sqrt(np.mean(G ** 2)))
     dU = 8e-3 * np.abs(U) + 1e-3 * float(np.sqrt(np.mean(U ** 2)))
-    return 1.1 * np.abs(U) * dG + np.abs(silu(G)) * dU
+    L = max_abs_silu_prime(G - dG, G + dG)
+    band = L * dG * (np.abs(U) + dU) + np.abs(silu(G)) * dU
+    if rel_eval:
+        band = band + rel_eval * (np.abs(silu(G)) + L * dG) * (np.abs(U) + dU)
+    return band
 
 
 def _scale_code(amax: np.ndarray, t: float) -> np.ndarray:

@@ -420,6 +420,72 @@ def test_consistency_check_accepts_both_sides_of_a_threshold_inside_the_band():
     assert not swiglu.consistent(up, scales, H, np.zeros_like(H), t)[0]
 
 
+def _band_cases(seed):
+    """G, U covering the regimes of silu: around 0, around the zero of silu'
+    (g = -1.2785), around the extrema of silu' (g = +-2.3994), far negative,
+    far positive, and U near zero; plus typical N(0, 3) pairs."""
+    rng = np.random.default_rng(seed)
+    centres = [0.0, -1.278464542761074, -2.3993572805154675, 2.3993572805154675, -12.0, 15.0, 0.3]
+    G = np.concatenate([c + rng.normal(0, 0.05, 60) for c in centres] + [rng.normal(0, 3, 400)])
+    U = np.concatenate([rng.normal(0, 2, 60 * len(centres) - 100), rng.normal(0, 1e-3, 100),
+                        rng.normal(0, 3, 400)])
+    U[:20] = 0.0
+    G[-20:] = 0.0
+    return G[None, :], U[None, :]
+
+
+def _brute_band(G, U, n=801):
+    """max over g' on a grid of [G - dG, G + dG] (ends and silu's critical
+    point included) and u' in {U - dU, U + dU} of |silu(g') u' - silu(G) U|."""
+    from oracle import swiglu
+    dG = 8e-3 * np.abs(G) + 1e-3 * np.sqrt(np.mean(G ** 2))
+    dU = 8e-3 * np.abs(U) + 1e-3 * np.sqrt(np.mean(U ** 2))
+    f = np.linspace(-1.0, 1.0, n)[:, None, None]
+    gp = G[None] + f * dG[None]
+    crit = np.full_like(G, -1.278464542761074)
+    inside = (G - dG <= crit) & (crit <= G + dG)
+    gp = np.concatenate([gp, np.where(inside, crit, G)[None]], axis=0)
+    h0 = swiglu.silu(G) * U
+    best = np.zeros_like(G)
+    for up in (U - dU, U + dU):
+        best = np.maximum(best, np.max(np.abs(swiglu.silu(gp) * up[None] - h0[None]), axis=0))
+    return best
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_silu_mul_error_band_covers_brute_force_and_is_tight(seed):
+    """The acceptance band of the SiLU * mul epilogue, pinned by brute force
+    over the GEMM bar of G and U: it must contain every |H' - H| reachable
+    there, and be at most about twice the largest of them."""
+    from oracle import swiglu
+    G, U = _band_cases(seed)
+    band = swiglu.error_band(G, U)
+    brute = _brute_band(G, U)
+    assert np.all(band >= brute * (1 - 1e-9)), float(np.max(brute / np.maximum(band, 1e-300)))
+    ratio = band / np.maximum(brute, 1e-300)
+    assert np.all((ratio <= 2.05) | (band == 0)), float(np.max(ratio))
+    # the evaluation term only widens the band, by the stated relative amount at most
+    wide = swiglu.error_band(G, U, rel_eval=1e-5)
+    assert np.all(wide >= band)
+    assert np.all(wide - band <= 1e-5 * (np.abs(swiglu.silu(G)) + 1.1 * 0.5 * np.abs(G) + 1.0) * (np.abs(U) + 1.0))
+
+
+def test_silu_prime_bound_matches_dense_search():
+    """max |silu'| over an interval, from its ends and the two extrema of silu',
+    against a dense search."""
+    from oracle import swiglu
+    rng = np.random.default_rng(3)
+    lo = rng.uniform(-8, 8, 300)
+    hi = lo + rng.uniform(0, 4, 300)
+    dense = np.max(np.abs(swiglu.silu_prime(lo[None] + np.linspace(0, 1, 20001)[:, None] * (hi - lo)[None])), axis=0)
+    got = swiglu.max_abs_silu_prime(lo, hi)
+    assert np.all(got >= dense * (1 - 1e-12))
+    assert np.all(got <= dense * (1 + 1e-7))
+    # the extrema are where silu'' vanishes: about -0.0998 and +1.0998
+    vals = [float(swiglu.silu_prime(c)) for c in swiglu.SILU_PRIME_EXTREMA]
+    assert abs(vals[0] + 0.09984) < 1e-4 and abs(vals[1] - 1.09984) < 1e-4
+
+
 # ------------------------------------------------------------------ 2:4 sparse INT4 (oracle/sparse24.py)
 
 def test_prune24_keeps_two_largest_per_run_with_lower_index_on_ties():
