@@ -200,10 +200,11 @@ def scales_bytes(rows: int, K: int) -> int:
     return padded_rows(rows) * (K // BLOCK)
 
 
-def scale_offsets(rows: int, K: int) -> np.ndarray:
-    """Byte offset of logical scale (r, kb) in the tiled buffer, shape [rows, K/16]."""
+def scale_offsets(rows: int, K: int, row_index=None) -> np.ndarray:
+    """Byte offset of logical scale (r, kb) in the tiled buffer, shape [rows, K/16]
+    (or [len(row_index), K/16] for the listed rows only)."""
     assert K % 64 == 0
-    r = np.arange(rows)[:, None]
+    r = (np.arange(rows) if row_index is None else np.asarray(row_index, dtype=np.int64))[:, None]
     kb = np.arange(K // BLOCK)[None, :]
     atoms_per_row_tile = K // 64
     atom = (r // 128) * atoms_per_row_tile + kb // 4
