@@ -37,6 +37,7 @@ PREFILL_M = 8192
 DECODE_BATCHES = (1, 4, 8, 16, 32)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_OVER_BF16 = 4.0     # nominal dense ratio: 9 PF NVFP4 / 2.25 PF BF16
+QUANTIZE_LAUNCHES = 2   # kernels per nvfp4_quantize call with a computed tensor scale (amax pass, quantize)
 
 
 def rank_seed(base: int, layer: int, rank: int) -> int:
@@ -239,6 +240,35 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ GPU arm
+def fp4_peaks(peaks):
+    """Dense NVFP4 peaks (burst, sustained) in TFLOP/s: the measured BF16 cuBLAS
+    figures times the nominal dense FP4 / BF16 ratio."""
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP4_OVER_BF16
+    sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP4_OVER_BF16
+    return burst, sust
+
+
+def pick_fp4_peak(burst: float, sustained: float, clock_reasons):
+    """The burst peak applies unless the run's own clock record shows the power
+    cap (the sustained figure was measured under it)."""
+    if "sw_power_cap" in (clock_reasons or []):
+        return sustained, "sustained (sw_power_cap seen during the timed region)"
+    return burst, "burst (no sw_power_cap during the timed region)"
+
+
+def mean_sd(vals):
+    vals = [float(v) for v in vals]
+    m = statistics.fmean(vals)
+    sd = statistics.stdev(vals) if len(vals) > 1 else 0.0
+    return m, sd
+
+
+def split_steps(steps: int, repeats: int):
+    """K timed steps as `repeats` contiguous blocks (sizes differ by at most one)."""
+    repeats = max(1, min(repeats, steps))
+    return [steps // repeats + (1 if r < steps % repeats else 0) for r in range(repeats)]
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -290,7 +320,7 @@ def run_gpu(args):
             wsb = nvq.w4a16_workspace_bytes(M, N, K)
             dec.append(dict(M=M, K=K, N=N, layer=i, x=x, pc=dec_w[mi][i][0], ps=dec_w[mi][i][1],
                             y=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
-                            ws=torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)))
+                            ws=torch.zeros(max(wsb, 16), dtype=torch.uint8, device=dev)))
     torch.cuda.synchronize()
 
     # external=True: the records become timestamp nodes of the captured graph
@@ -323,7 +353,7 @@ def run_gpu(args):
                     nvq.w4a16_gemm(D["x"], D["pc"], D["ps"], D["N"], y=D["y"], workspace=D["ws"], stream=stream)
             db.record(stream)
 
-    launches_per_step = 3 * len(pre) + len(dec)
+    launches_per_step = QUANTIZE_LAUNCHES * len(pre) + len(pre) + len(dec)
     step()                                  # first calls set kernel attributes outside capture
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
@@ -331,30 +361,53 @@ def run_gpu(args):
         step()
     torch.cuda.synchronize()
 
+    def replay_and_read():
+        """One step; its per-kernel device times (ms) from the graph's event nodes."""
+        graph.replay()
+        stream.synchronize()
+        return (pre_ev[0].elapsed_time(pre_ev[1]),
+                sum(a.elapsed_time(b) for a, b in g_ev),
+                sum(a.elapsed_time(b) for a, b in q_ev),
+                d_ev[0][0].elapsed_time(d_ev[0][1]),
+                d_ev[1][0].elapsed_time(d_ev[1][1]),
+                [a.elapsed_time(b) for a, b in g_ev])
+
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()
 
+    # ---------------- noise sizing: two identical conditions, interleaved
+    noise = None
+    if rank == 0 or world > 1:
+        blocks = {"A": [], "B": []}
+        for b in range(6):
+            vals = [replay_and_read()[0] for _ in range(10)]
+            blocks["A" if b % 2 == 0 else "B"].append(statistics.fmean(vals))
+        (ma, sa), (mb, sb) = mean_sd(blocks["A"]), mean_sd(blocks["B"])
+        noise = {"what": "the same prefill pass timed as two conditions A and B, 3 interleaved blocks of "
+                         "10 steps each", "A_ms": ma, "A_sd_ms": sa, "B_ms": mb, "B_sd_ms": sb,
+                 "diff_pct": 100.0 * abs(ma - mb) / ma}
+
     smi_id = gpu_smi_id(torch, local)
     t_start, t_end = ev(), ev()
-    q_ms = [0.0] * len(pre)
-    g_ms = [0.0] * len(pre)
-    d_ms = [0.0] * len(d_ev)
-    pre_ms = 0.0
+    reps = {"pass": [], "gemm": [], "quant": [], "dec16": [], "dec32": []}
+    g_layer = [0.0] * len(pre)
+    sizes = split_steps(args.steps, args.repeats)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(smi_id) as clocks:
         t_start.record(stream)
-        for _ in range(args.steps):
-            graph.replay()
-            stream.synchronize()                # read this replay's kernel events
-            pre_ms += pre_ev[0].elapsed_time(pre_ev[1])
-            for j in range(len(pre)):
-                q_ms[j] += q_ev[j][0].elapsed_time(q_ev[j][1])
-                g_ms[j] += g_ev[j][0].elapsed_time(g_ev[j][1])
-            for j in range(len(d_ev)):
-                d_ms[j] += d_ev[j][0].elapsed_time(d_ev[j][1])
+        for n in sizes:
+            acc = [0.0] * 5
+            for _ in range(n):
+                r = replay_and_read()
+                for j in range(5):
+                    acc[j] += r[j]
+                for j in range(len(pre)):
+                    g_layer[j] += r[5][j]
+            for key, v in zip(reps, acc):
+                reps[key].append(v / n)
         t_end.record(stream)
         torch.cuda.synchronize()
     total_ms = t_start.elapsed_time(t_end)
@@ -364,27 +417,23 @@ def run_gpu(args):
 
     K_steps = args.steps
     gemm_flops = sum(2.0 * PREFILL_M * L["N"] * L["K"] for L in pre)
-    pre_s = pre_ms / 1e3 / K_steps
-    gemm_s = sum(g_ms) / 1e3 / K_steps
-    quant_s = sum(q_ms) / 1e3 / K_steps
+    pass_m, pass_sd = mean_sd(reps["pass"])
+    gemm_m, gemm_sd = mean_sd(reps["gemm"])
+    quant_m, quant_sd = mean_sd(reps["quant"])
+    d16_m, d16_sd = mean_sd(reps["dec16"])
 
     def dec_bytes(D):
         M, K, N = D["M"], D["K"], D["N"]
         return N * K / 2 + 2 * N * K / 128 + 2 * M * K + 2 * M * N
 
     dec_b = sum(dec_bytes(D) for D in dec if D["M"] <= 16)
-    dec_s = d_ms[0] / 1e3 / K_steps
+    # max over ranks of the step time and of the per-kernel means
+    total_ms, pass_m, gemm_m, d16_m = max_over_ranks(torch, dist if world > 1 else None,
+                                                     [total_ms, pass_m, gemm_m, d16_m], dev)
+    gemm_tflops = gemm_flops / (gemm_m / 1e3) / 1e12      # per GPU (slowest rank): the kernel's roofline
+    value = whole_job_rate(gemm_flops, world, pass_m / 1e3) / 1e12
+    dec_gbs = dec_b / (d16_m / 1e3) / 1e9
     per_batch = per_batch_decode(torch, nvq, dec, dec_w, stream, dec_bytes)
-
-    peaks, peaks_kind = load_peaks()
-    fp4_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP4_OVER_BF16
-    fp4_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP4_OVER_BF16
-    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    # max over ranks of the step time and of the per-kernel sums
-    total_ms, pre_s, gemm_s, dec_s = max_over_ranks(torch, dist if world > 1 else None,
-                                                    [total_ms, pre_s, gemm_s, dec_s], dev)
-    gemm_tflops = gemm_flops / gemm_s / 1e12          # per GPU (slowest rank): the kernel's roofline
-    value = whole_job_rate(gemm_flops, world, pre_s) / 1e12
 
     # ---------------- end to end through the public API with host buffers
     e2e = None
@@ -393,8 +442,21 @@ def run_gpu(args):
     if world > 1:
         e2e["seconds"] = max_over_ranks(torch, dist, [e2e["seconds"]], dev)[0]
 
+    peaks, peaks_kind = load_peaks()
+    fp4_burst, fp4_sust = fp4_peaks(peaks)
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    extra = {}
+    if rank == 0 and not args.no_extra:
+        del pre, dec, dec_w
+        torch.cuda.empty_cache()
+        extra["config4"] = measure_config4(torch, nvq, synth, stream, dev, fp4_burst, fp4_sust, args.repeats)
+        extra["crossover"] = measure_crossover(torch, nvq, synth, stream, dev, args.repeats)
+
     if rank == 0:
         clk = clocks.summary()
+        fp4_peak, peak_rule = pick_fp4_peak(fp4_burst, fp4_sust, clk["reasons"])
+        layer_tflops = {LINEARS[j][0]: 2.0 * PREFILL_M * LINEARS[j][2] * LINEARS[j][1] /
+                        (g_layer[j] / K_steps / 1e3) / 1e12 for j in range(len(LINEARS))}
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K_steps,
             "warmup": args.warmup, "ms_per_step": total_ms / K_steps, "higher_is_better": True,
@@ -405,24 +467,30 @@ def run_gpu(args):
                        "seq_len": PREFILL_M, "linears": [list(l) for l in LINEARS],
                        "l2": "inputs larger than L2 (prefill pass touches ~1.3 GB; five decode weight copies)",
                        "parallelism": f"independent per-rank workloads x{world}"},
-            "prefill": {"gemm_only_tflops": gemm_tflops, "quantize_ms": 1e3 * quant_s, "gemm_ms": 1e3 * gemm_s,
-                        "pass_ms": 1e3 * pre_s,
-                        "per_layer_gemm_tflops": {L["name"]: 2.0 * PREFILL_M * L["N"] * L["K"] /
-                                                  (g_ms[j] / 1e3 / K_steps) / 1e12 for j, L in enumerate(pre)}},
+            "protocol": {"repeats": len(sizes), "steps_per_repeat": sizes,
+                         "interleaved": "each step runs the prefill pass then the decode blocks",
+                         "noise": noise},
+            "prefill": {"pass_ms": pass_m, "pass_sd_ms": pass_sd,
+                        "gemm_ms": gemm_m, "gemm_sd_ms": gemm_sd,
+                        "quantize_ms": quant_m, "quantize_sd_ms": quant_sd,
+                        "gemm_only_tflops": gemm_tflops,
+                        "per_layer_gemm_tflops": layer_tflops},
             "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_kernel", "achieved": gemm_tflops,
                          "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
-                         "peak_source": f"{peaks_kind} bf16 sustained x 4 (nominal FP4/BF16 dense ratio)",
+                         "peak_source": f"{peaks_kind} bf16 x 4 (nominal FP4/BF16 dense ratio), {peak_rule}",
                          "frac_of_burst_peak": gemm_tflops / fp4_burst,
+                         "frac_of_sustained_peak": gemm_tflops / fp4_sust,
                          "traffic": profiled_traffic("nvfp4_gemm_qwen3_8b_prefill.md", "nvfp4_gemm.cuh")},
-            "decode": {"metric": "INT4 W-only decode GB/s (M <= 16)", "value": dec_b / dec_s / 1e9,
-                       "unit": "GB/s", "per_batch": per_batch,
-                       "roofline": {"bound": "hbm", "kernel": "w4a16_kernel", "achieved": dec_b / dec_s / 1e9,
-                                    "peak": hbm, "unit": "GB/s", "frac": dec_b / dec_s / 1e9 / hbm,
+            "decode": {"metric": "INT4 W-only decode GB/s (M <= 16)", "value": dec_gbs, "unit": "GB/s",
+                       "block_ms": d16_m, "block_sd_ms": d16_sd, "per_batch": per_batch,
+                       "roofline": {"bound": "hbm", "kernel": "w4a16_kernel", "achieved": dec_gbs,
+                                    "peak": hbm, "unit": "GB/s", "frac": dec_gbs / hbm,
                                     "peak_source": f"{peaks_kind} copy bandwidth",
                                     "traffic": profiled_traffic("w4a16_decode_qwen3_8b.md", "w4a16_gemm.cuh")}},
             "clocks": clk,
             "gpu_launches": launches_per_step * K_steps,
         }
+        line.update(extra)
         line["e2e"] = {"value": world * gemm_flops / e2e["seconds"] / 1e12, "unit": "TFLOP/s",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
         if world == 1:
@@ -433,6 +501,134 @@ def run_gpu(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def graph_layer_times(torch, stream, calls, reps):
+    """Capture `calls` (a list of no-argument launchers) in one graph with an
+    event pair around each; replay it `reps` times.  Returns per-call lists of
+    device milliseconds (one entry per replay)."""
+    ev = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
+    evs = [(ev(), ev()) for _ in calls]
+
+    def run():
+        for (a, b), c in zip(evs, calls):
+            a.record(stream)
+            c()
+            b.record(stream)
+
+    run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        run()
+    g.replay()
+    torch.cuda.synchronize()
+    out = [[] for _ in calls]
+    for _ in range(reps):
+        g.replay()
+        stream.synchronize()
+        for i, (a, b) in enumerate(evs):
+            out[i].append(a.elapsed_time(b))
+    del g
+    return out
+
+
+def measure_config4(torch, nvq, synth, stream, dev, fp4_burst, fp4_sust, repeats):
+    """Qwen3-32B prefill linears at M = 32768 tokens: the W4A4 GEMM of each
+    layer, inputs quantized once beforehand (untimed), every operand larger
+    than L2.  One graph of the four GEMMs replayed `repeats` times."""
+    M = 32768
+    layers = []
+    for i, (name, K, N) in enumerate(synth.QWEN3_32B_LINEARS):
+        x = synth.activations_cuda(M, K, seed=4000 + 10 * i, device=dev)
+        w = synth.weights_cuda(N, K, seed=4000 + 10 * i, device=dev)
+        xq, wq = nvq.nvfp4_quantize(x), nvq.nvfp4_quantize(w)
+        del x, w
+        layers.append(dict(name=name, K=K, N=N, xq=xq, wq=wq,
+                           y=torch.empty(M, N, dtype=torch.bfloat16, device=dev)))
+    torch.cuda.synchronize()
+    calls = [(lambda L=L: nvq.nvfp4_gemm_w4a4(L["xq"], L["wq"], M, L["N"], L["K"], y=L["y"], stream=stream))
+             for L in layers]
+    with ClockSampler(gpu_smi_id(torch, dev.index)) as clocks:
+        times = graph_layer_times(torch, stream, calls, max(repeats, 5))
+    nvq.check_device_error(stream)
+    clk = clocks.summary()
+    peak, rule = pick_fp4_peak(fp4_burst, fp4_sust, clk["reasons"])
+    out = {"workload": "Qwen3-32B prefill linears, M=32768 tokens, NVFP4 W4A4 GEMM (quantized inputs resident)",
+           "repeats": len(times[0]), "peak": peak, "peak_rule": rule, "clocks": clk, "layers": {}}
+    flops_all, ms_all = 0.0, 0.0
+    for L, t in zip(layers, times):
+        m, sd = mean_sd(t)
+        fl = 2.0 * M * L["N"] * L["K"]
+        tf = fl / (m / 1e3) / 1e12
+        flops_all += fl
+        ms_all += m
+        out["layers"][L["name"]] = {"K": L["K"], "N": L["N"], "ms": m, "sd_ms": sd, "tflops": tf,
+                                    "frac": tf / peak, "frac_of_burst_peak": tf / fp4_burst}
+    out["tflops"] = flops_all / (ms_all / 1e3) / 1e12
+    out["frac"] = out["tflops"] / peak
+    out["frac_of_burst_peak"] = out["tflops"] / fp4_burst
+    del layers
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_crossover(torch, nvq, synth, stream, dev, repeats, copies=4):
+    """The phase crossover on the gate_up shape (K = 4096, N = 24576): one BF16
+    master weight quantized both ways (NVFP4 for W4A4, INT4 g128 for W4A16),
+    both paths timed at every M.  Each graph cycles through `copies` copies of
+    the weights (about 210-230 MB, above L2), so weights come from HBM; the
+    W4A4 path includes the activation quantize (amax + codes)."""
+    K, N = 4096, 24576
+    Mmax = max(synth.CROSSOVER_BATCHES)
+    w = synth.weights_cuda(N, K, seed=5000, device=dev)
+    wq = nvq.nvfp4_quantize(w)
+    codes, scales = nvq.int4_quantize(w)
+    pc, ps = nvq.int4_pack_weights(codes, scales, N, K)
+    del w, codes, scales
+    wq_c = [tuple(t.clone() for t in wq) for _ in range(copies)]
+    pk_c = [(pc.clone(), ps.clone()) for _ in range(copies)]
+    xc = torch.empty(Mmax, K // 2, dtype=torch.uint8, device=dev)
+    xs = torch.empty(nvq.nvfp4_scales_bytes(Mmax, K), dtype=torch.uint8, device=dev)
+    tx = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = torch.empty(nvq.nvfp4_quantize_workspace_bytes(Mmax, K), dtype=torch.uint8, device=dev)
+    y = torch.empty(Mmax * N, dtype=torch.bfloat16, device=dev)
+    dws = torch.zeros(max(16, nvq.w4a16_workspace_bytes(Mmax, N, K)), dtype=torch.uint8, device=dev)
+    out = {"workload": "gate_up K=4096 N=24576, weights cycled through 4 copies (from HBM)",
+           "repeats": max(repeats, 5), "per_M": {}}
+    faster16 = []
+    for M in synth.CROSSOVER_BATCHES:
+        x = synth.activations_cuda(M, K, seed=5000 + M, device=dev)
+        yM = y[:M * N].view(M, N)
+        sb = nvq.nvfp4_scales_bytes(M, K)
+
+        def w16(i, x=x, yM=yM):
+            p = pk_c[i % copies]
+            nvq.w4a16_gemm(x, p[0], p[1], N, y=yM, workspace=dws, stream=stream)
+
+        def w4(i, x=x, yM=yM, M=M, sb=sb):
+            q = (xc[:M], xs[:sb], tx)
+            nvq.nvfp4_quantize(x, None, codes=q[0], scales=q[1], tensor_scale_out=tx, workspace=ws, stream=stream)
+            nvq.nvfp4_gemm_w4a4(q, wq_c[i % copies], M, N, K, y=yM, stream=stream)
+
+        res = {}
+        for name, fn in (("w4a16", w16), ("w4a4", w4)):
+            ncall = 2 * copies
+            t = graph_layer_times(torch, stream, [lambda fn=fn: [fn(i) for i in range(ncall)]],
+                                  out["repeats"])[0]
+            m, sd = mean_sd([v / ncall for v in t])
+            res[name + "_us"] = 1e3 * m
+            res[name + "_sd_us"] = 1e3 * sd
+        res["faster"] = "w4a16" if res["w4a16_us"] < res["w4a4_us"] else "w4a4"
+        if res["faster"] == "w4a16":
+            faster16.append(M)
+        out["per_M"][str(M)] = res
+        del x
+    nvq.check_device_error(stream)
+    out["w4a16_faster_up_to_M"] = max(faster16) if faster16 else 0
+    del wq_c, pk_c, xc, xs, y
+    torch.cuda.empty_cache()
+    return out
 
 
 def per_batch_decode(torch, nvq, dec, dec_w, stream, dec_bytes, reps: int = 20):
@@ -532,6 +728,8 @@ def main():
                     help="timed steps (default: 400 on the GPU, about one second; 20 for the CPU oracle arm)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="nvq", choices=("nvq", "reference"))
+    ap.add_argument("--repeats", type=int, default=5, help="timed steps are split into this many repeats (mean, sd)")
+    ap.add_argument("--no-extra", action="store_true", help="skip the Qwen3-32B and crossover measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

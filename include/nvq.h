@@ -343,7 +343,7 @@ nvq_status w4a16_sparse24_gemm(const void* x_bf16, const uint8_t* packed, const 
  * crossover_m < 0 selects nvq_default_crossover_m(): the largest M at which
  * the W4A16 path was measured faster than quantize + W4A4 on B200 for the
  * Qwen3-8B gate_up shape (K = 4096, N = 24576), weights read from HBM
- * (python -m phase_disaggregated_quantized_b200.profile_case --op crossover).
+ * (python profile_case.py --op crossover).
  * workspace: nvq_linear_workspace_bytes(M, N, K, crossover_m) bytes, 16-byte
  * aligned (activation codes, scales, t and the quantizer's scratch), NULL when
  * that is 0.  Output y_bf16 [M, N] BF16, row stride N.

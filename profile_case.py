@@ -1,11 +1,11 @@
 """Run one library call on one shape a few times, for profilers (ncu) and quick timing.
 
-  python -m phase_disaggregated_quantized_b200.profile_case --op gemm --M 8192 --K 4096 --N 24576
-  python -m phase_disaggregated_quantized_b200.profile_case --op w4a16 --M 1 --K 4096 --N 24576
-  python -m phase_disaggregated_quantized_b200.profile_case --op quantize --M 8192 --K 12288
-  python -m phase_disaggregated_quantized_b200.profile_case --op crossover --K 4096 --N 24576
-  python -m phase_disaggregated_quantized_b200.profile_case --op streamed --M 8192 --layers 8
-  python -m phase_disaggregated_quantized_b200.profile_case --op swiglu --M 8192 --K 4096 --N 24576
+  python profile_case.py --op gemm --M 8192 --K 4096 --N 24576
+  python profile_case.py --op w4a16 --M 1 --K 4096 --N 24576
+  python profile_case.py --op quantize --M 8192 --K 12288
+  python profile_case.py --op crossover --K 4096 --N 24576
+  python profile_case.py --op streamed --M 8192 --layers 8
+  python profile_case.py --op swiglu --M 8192 --K 4096 --N 24576
 
 Inputs are drawn on the GPU from the seeded generators; the offline steps
 (weight quantization and reorder) run once before the measured calls.  The
@@ -17,11 +17,14 @@ bytes than L2 holds (126 MB).
 from __future__ import annotations
 
 import argparse
+import os
+import sys
 
 import torch
 
-import phase_disaggregated_quantized_b200 as nvq
-from phase_disaggregated_quantized_b200 import synth
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+import phase_disaggregated_quantized_b200 as nvq  # noqa: E402
+from phase_disaggregated_quantized_b200 import synth  # noqa: E402
 
 
 def main():

@@ -53,3 +53,20 @@ def test_committed_profiles_name_a_traffic_figure_for_both_hot_kernels():
         text = open(os.path.join(ROOT, "profiles", summary)).read()
         assert "traffic_source_hash:" in text and "traffic_bytes_per_launch:" in text
         assert os.path.exists(os.path.join(ROOT, "phase_disaggregated_quantized_b200", "csrc", source))
+
+
+def test_fp4_peak_is_burst_unless_the_power_cap_was_seen():
+    burst, sust = bench.fp4_peaks({"bf16_tflops": 1627.0, "bf16_tflops_sustained": 1401.6})
+    assert burst == 1627.0 * 4 and sust == 1401.6 * 4
+    assert bench.pick_fp4_peak(burst, sust, [])[0] == burst
+    assert bench.pick_fp4_peak(burst, sust, ["hw_slowdown"])[0] == burst
+    assert bench.pick_fp4_peak(burst, sust, ["sw_power_cap"])[0] == sust
+
+
+def test_timed_steps_split_into_repeats():
+    assert bench.split_steps(400, 5) == [80] * 5
+    assert bench.split_steps(12, 5) == [3, 3, 2, 2, 2]
+    assert sum(bench.split_steps(7, 5)) == 7
+    assert bench.split_steps(3, 5) == [1, 1, 1]
+    m, sd = bench.mean_sd([1.0, 2.0, 3.0])
+    assert m == 2.0 and abs(sd - 1.0) < 1e-12
