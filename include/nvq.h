@@ -62,9 +62,8 @@ const char* nvq_last_error_detail(void);
 
 /* Workspace bytes of one call, by operation (the per-operation *_workspace_bytes
  * functions give the same numbers): NVQ_OP_NVFP4_QUANTIZE (rows = M, K; also
- * nvfp4_amax), NVQ_OP_NVFP4_GEMM (0: none), NVQ_OP_W4A16_GEMM (tile tickets
- * and partial tiles for M <= 32, 0 above), NVQ_OP_LINEAR (nvq_linear at the
- * default crossover).
+ * nvfp4_amax), NVQ_OP_NVFP4_GEMM (0: none), NVQ_OP_W4A16_GEMM (0: partial sums
+ * stay on chip), NVQ_OP_LINEAR (nvq_linear at the default crossover).
  * SIZE_MAX for an unknown op. */
 typedef enum {
   NVQ_OP_NVFP4_QUANTIZE = 0,
@@ -282,19 +281,9 @@ nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int6
  *
  * x_bf16 [M, K] BF16; packed_codes / packed_scales from int4_pack_weights;
  * y_bf16 [M, N] BF16, row stride N, written.
- * For M <= 32 (one batch tile: the decode case) the weight units are split
- * evenly over every CTA of the grid, and the few 32-row output tiles that a
- * CTA boundary cuts are finished through the workspace: one 4-byte ticket
- * counter per tile, then two partial-tile slots per CTA.  workspace: at least
- * w4a16_workspace_bytes(M, N, K) bytes (it depends on N, on M only through
- * M <= 8 / 16 / 32, and on the current device's SM count), 16-byte aligned,
- * filled with zeros before its first use; every call leaves the counters at
- * zero again, so one workspace serves any number of calls on one stream.  Two
- * calls that may run at the same time (different streams) need different
- * workspaces.  After NVQ_ERR_DEVICE_TIMEOUT zero it again.
- * NVQ_ERR_WORKSPACE if it is missing or too small.  For M > 32 the workspace
- * is not used (w4a16_workspace_bytes returns 0): clusters of CTAs own whole
- * tiles and process the batch 32 rows per pass over W.
+ * workspace / workspace_bytes: unused (w4a16_workspace_bytes returns 0, the
+ * partial sums stay on chip); kept so callers need not change.
+ * Runs best for M <= 16; larger M is processed 32 rows per pass over W.
  * Launched with programmatic dependent launch: the call may begin while the
  * preceding kernel on the stream is still finishing, and it starts streaming
  * the packed weights before waiting for that kernel (x and y are touched only
@@ -330,16 +319,13 @@ nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const voi
  *
  * w4a16_sparse24_gemm: Y = X (s (u - 8) at the kept positions, 0 elsewhere)^T,
  * with the arithmetic of w4a16_gemm (exact products, FP32 sums, group scale in
- * FP32, BF16 RNE out) and its streaming kernel on 24% fewer weight bytes;
- * workspace as for w4a16_gemm (w4a16_workspace_bytes(M, N, K) bytes, zeroed
- * before first use, left zeroed by every call).
+ * FP32, BF16 RNE out) and its streaming kernel on 24% fewer weight bytes.
  * Shape rules for both: N % 32 == 0, K % 128 == 0; pointers 16-byte aligned.
  * ------------------------------------------------------------------------ */
 nvq_status int4_pack_sparse24(const void* w_bf16, const uint8_t* codes, const void* scales_bf16, int64_t N,
                               int64_t K, uint8_t* packed, void* packed_scales, void* stream);
 nvq_status w4a16_sparse24_gemm(const void* x_bf16, const uint8_t* packed, const void* packed_scales,
-                               void* y_bf16, int64_t M, int64_t N, int64_t K, void* workspace,
-                               size_t workspace_bytes, void* stream);
+                               void* y_bf16, int64_t M, int64_t N, int64_t K, void* stream);
 
 /* ------------------------------------------------------------------------ *
  * Phase dispatch over one master weight held in both formats (Disaggregated
@@ -359,12 +345,8 @@ nvq_status w4a16_sparse24_gemm(const void* x_bf16, const uint8_t* packed, const 
  * Qwen3-8B gate_up shape (K = 4096, N = 24576), weights read from HBM
  * (python profile_case.py --op crossover).
  * workspace: nvq_linear_workspace_bytes(M, N, K, crossover_m) bytes, 16-byte
- * aligned, zeroed before its first use: first the W4A16 path's region (as
- * w4a16_gemm's workspace, sized for M = 32 so it stays in place for every M;
- * left zeroed by each call), then, when M > crossover_m, the W4A4 path's
- * activation codes, scales, t and quantizer scratch.  A workspace sized for
- * the largest M serves every smaller M.  Output y_bf16 [M, N] BF16, row
- * stride N.
+ * aligned (activation codes, scales, t and the quantizer's scratch), NULL when
+ * that is 0.  Output y_bf16 [M, N] BF16, row stride N.
  * Shape rules: those of the chosen path (W4A16: N % 32 == 0, K % 128 == 0;
  * W4A4: N % 8 == 0, K % 64 == 0).  Errors as the underlying calls.
  * ------------------------------------------------------------------------ */

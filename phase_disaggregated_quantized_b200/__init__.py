@@ -81,7 +81,7 @@ def lib() -> ctypes.CDLL:
             "w4a16_workspace_bytes": ([i64, i64, i64], sz),
             "w4a16_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp, sz, vp], i32),
             "int4_pack_sparse24": ([vp, vp, vp, i64, i64, vp, vp, vp], i32),
-            "w4a16_sparse24_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp, sz, vp], i32),
+            "w4a16_sparse24_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp], i32),
             "nvq_default_crossover_m": ([], i64),
             "nvq_linear_workspace_bytes": ([i64, i64, i64, i64], sz),
             "nvq_linear": ([vp, i64, i64, i64, vp, vp, vp, vp, vp, i64, vp, vp, sz, vp], i32),
@@ -298,7 +298,7 @@ def w4a16_gemm(x, packed_codes, packed_scales, N: int, *, y=None, workspace=None
         y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
     need = w4a16_workspace_bytes(M, N, K)
     if workspace is None and need:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)   # tickets start at zero
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().w4a16_gemm(_ptr(x), _ptr(packed_codes), _ptr(packed_scales), _ptr(y), M, N, K, _ptr(workspace),
                             ws_bytes, _stream(stream)), "w4a16_gemm")
@@ -319,20 +319,15 @@ def int4_pack_sparse24(w, codes, scales, *, packed=None, packed_scales=None, str
     return packed, packed_scales
 
 
-def w4a16_sparse24_gemm(x, packed, packed_scales, N: int, *, y=None, workspace=None, stream=None):
-    """BF16 X [M, K] times the 2:4-sparse packed INT4 W [N, K] -> Y [M, N] bf16.
-    workspace: w4a16_workspace_bytes(M, N, K) bytes, zeroed before first use."""
+def w4a16_sparse24_gemm(x, packed, packed_scales, N: int, *, y=None, stream=None):
+    """BF16 X [M, K] times the 2:4-sparse packed INT4 W [N, K] -> Y [M, N] bf16."""
     _need_cuda(x, packed, packed_scales)
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
     M, K = x.shape
     if y is None:
         y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
-    need = w4a16_workspace_bytes(M, N, K)
-    if workspace is None and need:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().w4a16_sparse24_gemm(_ptr(x), _ptr(packed), _ptr(packed_scales), _ptr(y), M, N, K,
-                                     _ptr(workspace), ws_bytes, _stream(stream)), "w4a16_sparse24_gemm")
+    _check(lib().w4a16_sparse24_gemm(_ptr(x), _ptr(packed), _ptr(packed_scales), _ptr(y), M, N, K, _stream(stream)),
+           "w4a16_sparse24_gemm")
     return y
 
 
@@ -363,7 +358,7 @@ def nvq_linear(x, w4a4=None, w4a16=None, N: int | None = None, *, crossover_m: i
         y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
     need = nvq_linear_workspace_bytes(M, N, K, crossover_m)
     if workspace is None and need:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)   # decode tickets start at zero
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().nvq_linear(_ptr(x), M, N, K, _ptr(wc), _ptr(wsc), _ptr(wt), _ptr(pc), _ptr(ps), crossover_m,
                             _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)), "nvq_linear")

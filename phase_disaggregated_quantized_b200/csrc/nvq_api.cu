@@ -99,76 +99,16 @@ constexpr int64_t kMaxDim = (int64_t)1 << 31;
 constexpr int64_t kMaxBlocks = (int64_t)1 << 31;
 bool gemm_tiles_fit(int64_t M, int64_t N) { return ((M + 127) / 128) * ((N + 127) / 128) < kMaxBlocks; }
 
-// Decode launches.  Batch rows are handled 8 * NT8 at a time.
+// Decode launch: a persistent grid of clusters of nvq::w4a16::CS CTAs, as many
+// as can be resident at once (one CTA per SM), never more clusters than output
+// tiles (32 weight rows dense, 16 for 2:4 sparse).  Batch rows are handled 8 * NT8 at a time.
 constexpr int kMaxDevices = 64;
-constexpr int kDecodeMaxCtasPerSm = 2;
 
-size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
-
-// Decode with one batch tile (M <= 32): a persistent grid, as many CTAs as fit
-// at once (at most kDecodeMaxCtasPerSm per SM, never more than the units), the
-// units split evenly over all of them; tiles cut by a CTA boundary are summed
-// through the workspace: tile tickets (4 bytes per 32-row tile, 256-aligned),
-// then two partial-tile slots per CTA.
-int decode_tilef(int64_t M) { return 128 * 2 * (M <= 8 ? 1 : M <= 16 ? 2 : 4); }
-size_t decode_ws_bytes(int64_t M, int64_t N, int sms) {
-  if (M <= 0 || M > 32 || N <= 0) return 0;
-  return align256((size_t)(N / 32) * 4) + (size_t)2 * kDecodeMaxCtasPerSm * sms * decode_tilef(M) * sizeof(float);
-}
-
-template <int NT8, bool SPARSE>
-nvq_status launch_w4a16_flat(const void* x, const uint8_t* pc, const void* ps, void* y, int64_t M, int64_t N,
-                             int64_t K, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  using C = nvq::w4a16::Cfg<NT8, SPARSE>;
-  auto fn = nvq::w4a16::w4a16_kernel<NT8, SPARSE, true>;
-  static std::atomic<int> per_sm[kMaxDevices];   // 0: not queried yet on that device
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm: cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(NVQ_ERR_CUDA, "w4a16_gemm: device index out of range");
-  int bps = per_sm[dev].load(std::memory_order_acquire);
-  if (bps == 0) {                               // two threads may both get here: same result
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm: shared memory attribute");
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, fn, C::THREADS, C::SMEM);
-    if (e != cudaSuccess) return cuda_fail(e, "w4a16_gemm: occupancy query");
-    if (bps < 1) return fail(NVQ_ERR_CUDA, "w4a16_gemm: the decode kernel does not fit on this GPU");
-    bps = std::min(bps, kDecodeMaxCtasPerSm);
-    per_sm[dev].store(bps, std::memory_order_release);
-  }
-  const int sms = sm_count();
-  const int64_t ntiles = N / nvq::w4a16::Unit<SPARSE>::ROWS, units = ntiles * (K / 128);
-  const int64_t grid = std::min<int64_t>((int64_t)sms * bps, units);
-  const size_t cnt_bytes = align256((size_t)ntiles * 4);
-  const size_t need = cnt_bytes + (size_t)2 * grid * C::TILEF * sizeof(float);
-  if (workspace == nullptr || workspace_bytes < need)      // the caller checked w4a16_workspace_bytes(), >= need
-    return fail(NVQ_ERR_WORKSPACE, "w4a16_gemm: workspace missing or smaller than w4a16_workspace_bytes()");
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // may launch during the previous kernel's tail
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.gridDim = dim3((unsigned)grid, 1, 1);
-  cfg.blockDim = dim3(C::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = C::SMEM;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  e = cudaLaunchKernelEx(&cfg, fn, static_cast<const __nv_bfloat16*>(x), pc, static_cast<const uint8_t*>(ps),
-                         static_cast<__nv_bfloat16*>(y), (uint32_t)M, (uint32_t)N, (uint32_t)K,
-                         reinterpret_cast<uint32_t*>(ws), reinterpret_cast<float*>(ws + cnt_bytes));
-  if (e != cudaSuccess) return cuda_fail(e, "w4a16_kernel launch");
-  return launch_status("w4a16_kernel");
-}
-
-// Decode with several batch tiles (M > 32): a persistent grid of clusters of
-// nvq::w4a16::CS CTAs, as many as can be resident at once (one CTA per SM),
-// never more clusters than output tiles; each cluster owns whole 32-row tiles.
 template <int NT8, bool SPARSE = false>
 nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* y, int64_t M, int64_t N, int64_t K,
                         cudaStream_t stream) {
   using C = nvq::w4a16::Cfg<NT8, SPARSE>;
-  auto fn = nvq::w4a16::w4a16_kernel<NT8, SPARSE, false>;
+  auto fn = nvq::w4a16::w4a16_kernel<NT8, SPARSE>;
   static std::atomic<int> max_clusters[kMaxDevices];   // 0: not queried yet on that device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -202,8 +142,7 @@ nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* 
   cfg.gridDim = dim3((unsigned)(nclu * nvq::w4a16::CS), 1, 1);
   cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, fn, static_cast<const __nv_bfloat16*>(x), pc, static_cast<const uint8_t*>(ps),
-                         static_cast<__nv_bfloat16*>(y), (uint32_t)M, (uint32_t)N, (uint32_t)K,
-                         static_cast<uint32_t*>(nullptr), static_cast<float*>(nullptr));
+                         static_cast<__nv_bfloat16*>(y), (uint32_t)M, (uint32_t)N, (uint32_t)K);
   if (e != cudaSuccess) return cuda_fail(e, "w4a16_kernel launch");
   return launch_status("w4a16_kernel");
 }
@@ -213,6 +152,7 @@ nvq_status launch_w4a16(const void* x, const uint8_t* pc, const void* ps, void* 
 struct LinearWs {
   size_t codes, scales, t, scratch, total;
 };
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 LinearWs linear_ws_layout(int64_t M, int64_t K) {
   LinearWs L;
   L.codes = 0;
@@ -265,7 +205,7 @@ StreamWs stream_ws_layout(const nvq_stream_layer* layers, int n, int64_t M) {
 
 extern "C" {
 
-int nvq_abi_version(void) { return 2; }
+int nvq_abi_version(void) { return 1; }
 
 const char* nvq_status_string(nvq_status s) {
   switch (s) {
@@ -608,12 +548,16 @@ nvq_status int4_pack_weights(const uint8_t* codes, const void* scales_bf16, int6
 
 // ------------------------------------------------------------------ W4A16 decode GEMM
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  (void)M;
+  (void)N;
   (void)K;
-  return decode_ws_bytes(M, N, sm_count());
+  return 0;                                      // partial sums stay on chip
 }
 
 nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const void* packed_scales, void* y_bf16,
                       int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes, void* stream_) {
+  (void)workspace;
+  (void)workspace_bytes;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "w4a16_gemm: bad sizes");
   if (N % 32 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_gemm: need N % 32 == 0, K % 128 == 0");
@@ -623,17 +567,8 @@ nvq_status w4a16_gemm(const void* x_bf16, const uint8_t* packed_codes, const voi
   if (!x_bf16 || !packed_codes || !packed_scales || !y_bf16) return fail(NVQ_ERR_INVALID_ARG, "w4a16_gemm: NULL pointer");
   if (!aligned16(x_bf16) || !aligned16(packed_codes) || !aligned16(packed_scales) || !aligned16(y_bf16))
     return fail(NVQ_ERR_MISALIGNED, "w4a16_gemm: pointer not 16-byte aligned");
-  if (M <= 32) {
-    if (workspace == nullptr || workspace_bytes < decode_ws_bytes(M, N, sm_count()))
-      return fail(NVQ_ERR_WORKSPACE, "w4a16_gemm: workspace missing or smaller than w4a16_workspace_bytes()");
-    if (!aligned16(workspace)) return fail(NVQ_ERR_MISALIGNED, "w4a16_gemm: workspace not 16-byte aligned");
-  }
-  if (M <= 8) return launch_w4a16_flat<1, false>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, workspace,
-                                                 workspace_bytes, stream);
-  if (M <= 16) return launch_w4a16_flat<2, false>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, workspace,
-                                                  workspace_bytes, stream);
-  if (M <= 32) return launch_w4a16_flat<4, false>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, workspace,
-                                                  workspace_bytes, stream);
+  if (M <= 8) return launch_w4a16<1>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
+  if (M <= 16) return launch_w4a16<2>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
   return launch_w4a16<4>(x_bf16, packed_codes, packed_scales, y_bf16, M, N, K, stream);
 }
 
@@ -659,8 +594,7 @@ nvq_status int4_pack_sparse24(const void* w_bf16, const uint8_t* codes, const vo
 }
 
 nvq_status w4a16_sparse24_gemm(const void* x_bf16, const uint8_t* packed, const void* packed_scales, void* y_bf16,
-                               int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
-                               void* stream_) {
+                               int64_t M, int64_t N, int64_t K, void* stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (M < 0 || N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "w4a16_sparse24_gemm: bad sizes");
   if (N % 32 != 0 || K % 128 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "w4a16_sparse24_gemm: need N % 32 == 0, K % 128 == 0");
@@ -670,17 +604,8 @@ nvq_status w4a16_sparse24_gemm(const void* x_bf16, const uint8_t* packed, const 
   if (!x_bf16 || !packed || !packed_scales || !y_bf16) return fail(NVQ_ERR_INVALID_ARG, "w4a16_sparse24_gemm: NULL pointer");
   if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(packed_scales) || !aligned16(y_bf16))
     return fail(NVQ_ERR_MISALIGNED, "w4a16_sparse24_gemm: pointer not 16-byte aligned");
-  if (M <= 32) {
-    if (workspace == nullptr || workspace_bytes < decode_ws_bytes(M, N, sm_count()))
-      return fail(NVQ_ERR_WORKSPACE, "w4a16_sparse24_gemm: workspace missing or smaller than w4a16_workspace_bytes()");
-    if (!aligned16(workspace)) return fail(NVQ_ERR_MISALIGNED, "w4a16_sparse24_gemm: workspace not 16-byte aligned");
-  }
-  if (M <= 8) return launch_w4a16_flat<1, true>(x_bf16, packed, packed_scales, y_bf16, M, N, K, workspace,
-                                                workspace_bytes, stream);
-  if (M <= 16) return launch_w4a16_flat<2, true>(x_bf16, packed, packed_scales, y_bf16, M, N, K, workspace,
-                                                 workspace_bytes, stream);
-  if (M <= 32) return launch_w4a16_flat<4, true>(x_bf16, packed, packed_scales, y_bf16, M, N, K, workspace,
-                                                 workspace_bytes, stream);
+  if (M <= 8) return launch_w4a16<1, true>(x_bf16, packed, packed_scales, y_bf16, M, N, K, stream);
+  if (M <= 16) return launch_w4a16<2, true>(x_bf16, packed, packed_scales, y_bf16, M, N, K, stream);
   return launch_w4a16<4, true>(x_bf16, packed, packed_scales, y_bf16, M, N, K, stream);
 }
 
@@ -692,18 +617,11 @@ constexpr int64_t kDefaultCrossoverM = 16;
 
 int64_t nvq_default_crossover_m(void) { return kDefaultCrossoverM; }
 
-// nvq_linear's workspace: the W4A16 path's region (tile tickets + partial
-// slots, sized for the largest batch tile, so it never moves) first, then the
-// W4A4 path's activation quantizer outputs when M is above the crossover.  The
-// W4A4 path never writes the first region, so its tickets stay zero.
-size_t linear_decode_region(int64_t N) { return align256(decode_ws_bytes(32, N, sm_count())); }
-
 size_t nvq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t crossover_m) {
+  (void)N;
   if (crossover_m < 0) crossover_m = kDefaultCrossoverM;
-  if (M <= 0 || N <= 0 || K <= 0 || K % 64 != 0) return 0;
-  const size_t dec = linear_decode_region(N);
-  if (M <= crossover_m) return dec;
-  return dec + linear_ws_layout(M, K).total;
+  if (M <= crossover_m || M <= 0 || K <= 0 || K % 64 != 0) return 0;
+  return linear_ws_layout(M, K).total;
 }
 
 size_t nvq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
@@ -721,20 +639,17 @@ nvq_status nvq_linear(const void* x_bf16, int64_t M, int64_t N, int64_t K, const
                       const void* w_packed_scales, int64_t crossover_m, void* y_bf16, void* workspace,
                       size_t workspace_bytes, void* stream) {
   if (crossover_m < 0) crossover_m = kDefaultCrossoverM;
-  if (N <= 0 || K <= 0) return fail(NVQ_ERR_INVALID_ARG, "nvq_linear: bad sizes");
-  const size_t dec = linear_decode_region(N);
-  if (workspace != nullptr && !aligned16(workspace)) return fail(NVQ_ERR_MISALIGNED, "nvq_linear: workspace not 16-byte aligned");
   if (M <= crossover_m) {
     if (!w_packed_codes || !w_packed_scales) return fail(NVQ_ERR_INVALID_ARG, "nvq_linear: W4A16 path needs the packed INT4 weights");
-    return w4a16_gemm(x_bf16, w_packed_codes, w_packed_scales, y_bf16, M, N, K, workspace,
-                      workspace_bytes < dec ? workspace_bytes : dec, stream);
+    return w4a16_gemm(x_bf16, w_packed_codes, w_packed_scales, y_bf16, M, N, K, nullptr, 0, stream);
   }
   if (!w_codes || !w_scales || !w_t) return fail(NVQ_ERR_INVALID_ARG, "nvq_linear: W4A4 path needs the NVFP4 weights");
-  if (K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvq_linear: W4A4 path needs K % 64 == 0");
-  if (N % 8 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvq_linear: W4A4 path needs N % 8 == 0");
+  if (K <= 0 || K % 64 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvq_linear: W4A4 path needs K % 64 == 0");
+  if (N <= 0 || N % 8 != 0) return fail(NVQ_ERR_UNSUPPORTED_SHAPE, "nvq_linear: W4A4 path needs N % 8 == 0");
   const LinearWs L = linear_ws_layout(M, K);
-  if (workspace == nullptr || workspace_bytes < dec + L.total) return fail(NVQ_ERR_WORKSPACE, "nvq_linear: workspace too small");
-  uint8_t* ws = static_cast<uint8_t*>(workspace) + dec;
+  if (workspace == nullptr || workspace_bytes < L.total) return fail(NVQ_ERR_WORKSPACE, "nvq_linear: workspace too small");
+  if (!aligned16(workspace)) return fail(NVQ_ERR_MISALIGNED, "nvq_linear: workspace not 16-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint8_t* xc = ws + L.codes;
   uint8_t* xs = ws + L.scales;
   float* tx = reinterpret_cast<float*>(ws + L.t);

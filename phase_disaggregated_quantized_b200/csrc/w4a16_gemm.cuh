@@ -8,12 +8,10 @@
 // Work split.  The packed weights are a sequence of "units": one 128-wide
 // k-group of a tile of weight rows, tile-major.  Units hold 32 rows (two 16-row
 // MMA tiles): dense 2 KB of codes + 64 B of scales, 2:4-sparse 1536 B of codes
-// and metadata + 64 B of scales.  For one batch tile (M <= 32, the decode
-// case) the flat sequence is split evenly over all CTAs of the grid, and each
-// CTA's share evenly over its W warps, so every warp streams the same number
-// of bytes whatever N and K are (no whole-tile rounding).  For larger M each
-// cluster of CS CTAs owns a contiguous run of whole tiles and loops over the
-// batch in tiles of 8 NT8 rows, its units split over its CTAs and warps.
+// and metadata + 64 B of scales.  Each cluster of CS CTAs
+// owns a contiguous run of whole tiles; inside the cluster the run's units are
+// split evenly over CS CTAs x W warps, so every warp streams the same number of
+// bytes whatever N and K are.
 //
 // Streaming.  Each warp owns a ring of D stages of SG units in shared memory;
 // lane 0 refills a stage with two bulk copies (codes, scales) that complete on
@@ -32,16 +30,12 @@
 //
 // Reduction.  A warp writes tiles it covered entirely straight to Y; the tiles
 // at the ends of its range stay in registers and are summed by warp order in
-// shared memory.  Even split (one batch tile): a tile cut by a CTA boundary is
-// finished through a small global workspace -- each CTA that meets it stores
-// its partial in its own slot and takes a ticket from the tile's counter; the
-// CTA that draws the last ticket adds the slots in CTA order, writes Y and sets
-// the counter back to zero for the next call.  No CTA waits for another.
-// Clusters (several batch tiles): the one tile a cluster's two CTAs share is
-// finished by rank 1: rank 0 pushes its partial into rank 1's shared memory
-// with st.async, which completes on rank 1's mbarrier.  Either way the
-// summation order depends only on the shapes and the grid, so results are
-// reproducible run to run.
+// shared memory.  The one tile a cluster's two CTAs share (cut by their
+// boundary) is finished by rank 1: rank 0 pushes its partial into rank 1's
+// shared memory with st.async, which completes on rank 1's mbarrier, and rank 1
+// adds it before its own (rank order).  No cluster-wide barrier sits on the
+// exit path.  The summation order depends only on the shapes and the grid, so
+// results are reproducible run to run.
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
@@ -211,15 +205,6 @@ __device__ __forceinline__ uint32_t split_at(uint32_t len, uint32_t i) {
 }
 __host__ __device__ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v / 2); }
 
-// Even split of T units over C CTAs: CTA c owns [T c / C, T (c + 1) / C).
-__device__ __forceinline__ uint32_t flat_start(uint32_t T, uint32_t c, uint32_t C) {
-  return (uint32_t)(((uint64_t)T * c) / C);
-}
-// The CTA whose share holds unit u: the largest c with flat_start(c) <= u.
-__device__ __forceinline__ uint32_t flat_owner(uint32_t u, uint32_t T, uint32_t C) {
-  return (uint32_t)(((uint64_t)(u + 1) * C - 1) / T);
-}
-
 // Accumulator of one output tile: NTT = (16-row tiles) x (8-column batch tiles)
 // m16n8 fragments, fragment index tt * NT8 + t.
 template <int NTT>
@@ -239,14 +224,6 @@ __device__ __forceinline__ void add_tile(float (&a)[NTT][4], const float* p) {  
 #pragma unroll
   for (int t = 0; t < NTT; ++t) {
     const float4 v = *reinterpret_cast<const float4*>(p + 4 * t);
-    a[t][0] += v.x; a[t][1] += v.y; a[t][2] += v.z; a[t][3] += v.w;
-  }
-}
-template <int NTT>
-__device__ __forceinline__ void add_tile_l2(float (&a)[NTT][4], const float* p) {   // another CTA wrote p
-#pragma unroll
-  for (int t = 0; t < NTT; ++t) {
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(p + 4 * t));
     a[t][0] += v.x; a[t][1] += v.y; a[t][2] += v.z; a[t][3] += v.w;
   }
 }
@@ -396,16 +373,10 @@ __device__ __forceinline__ void sparse_unit(uint32_t unit, uint32_t lane, const 
   }
 }
 
-// FLAT: one batch tile (M <= 8 NT8), units split evenly over the whole grid
-// (no clusters), tiles cut by a CTA boundary finished through the workspace:
-// ws_cnt[ntiles] tickets (zero between calls), ws_slots[2 gridDim.x][TILEF]
-// partial tiles (slot 2c: CTA c's first tile, 2c + 1: its last).
-// !FLAT: clusters of CS CTAs own whole tiles and loop over batch tiles.
-template <int NT8, bool SPARSE, bool FLAT>
+template <int NT8, bool SPARSE>
 __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::MIN_CTAS) w4a16_kernel(
     const __nv_bfloat16* __restrict__ x, const uint8_t* __restrict__ pcodes, const uint8_t* __restrict__ pscales,
-    __nv_bfloat16* __restrict__ y, uint32_t M, uint32_t N, uint32_t K, uint32_t* __restrict__ ws_cnt,
-    float* __restrict__ ws_slots) {
+    __nv_bfloat16* __restrict__ y, uint32_t M, uint32_t N, uint32_t K) {
   using C = Cfg<NT8, SPARSE>;
   using U = typename C::U;
   constexpr uint32_t UC = U::CODE, USC = U::SCALE;
@@ -415,26 +386,16 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
   const uint32_t G = K >> 7, ntiles = N / U::ROWS;
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
   const uint32_t gl = lane >> 2;
+  const uint32_t rank = cluster_rank();
+  // This cluster's run of whole tiles, as flat units [A, A + L).
+  // Flat unit indices fit in 32 bits (the host rejects larger N * K).
   constexpr int LW = ilog2(W), LCS = ilog2(CS);
   static_assert((1 << LW) == W && (1 << LCS) == CS, "powers of two");
-  // This CTA's units [F0, F1).  Flat unit indices fit in 32 bits (the host
-  // rejects larger N * K).
-  uint32_t rank = 0, F0, F1;
-  if constexpr (FLAT) {
-    const uint32_t T = ntiles * G;
-    F0 = flat_start(T, blockIdx.x, gridDim.x);
-    F1 = flat_start(T, blockIdx.x + 1, gridDim.x);
-  } else {
-    // This cluster's run of whole tiles, as flat units [A, A + L).
-    rank = cluster_rank();
-    const uint32_t nclu = cluster_count(), cid = cluster_id();
-    const uint32_t tq = ntiles / nclu, tr = ntiles % nclu;
-    const uint32_t A = (tq * cid + tr * cid / nclu) * G;
-    const uint32_t L = (tq * (cid + 1) + tr * (cid + 1) / nclu) * G - A;
-    F0 = A + split_at<LCS>(L, rank);
-    F1 = A + split_at<LCS>(L, rank + 1);
-  }
-  const uint32_t FL = F1 - F0;
+  const uint32_t nclu = cluster_count(), cid = cluster_id();
+  const uint32_t tq = ntiles / nclu, tr = ntiles % nclu;
+  const uint32_t A = (tq * cid + tr * cid / nclu) * G;
+  const uint32_t L = (tq * (cid + 1) + tr * (cid + 1) / nclu) * G - A;
+  const uint32_t F0 = A + split_at<LCS>(L, rank), F1 = A + split_at<LCS>(L, rank + 1), FL = F1 - F0;   // this CTA
   const uint32_t f0 = F0 + split_at<LW>(FL, warp), f1 = F0 + split_at<LW>(FL, warp + 1);               // this warp
   const uint32_t nf = (uint32_t)(f1 - f0);
   const uint32_t sbase = smem_addr(smem);
@@ -444,11 +405,11 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
   const float* xslots = reinterpret_cast<const float*>(smem + C::XSLOT);
   const uint32_t rbar = sbase + C::XBARS, fbar = rbar + 16;   // [2] each, indexed by pass parity
   const uint64_t pol = policy_evict_first();
-  const uint32_t npass = FLAT ? 1u : (M + MC - 1) / MC;
+  const uint32_t npass = (M + MC - 1) / MC;
   static_assert(CS == 2, "the cross-CTA exchange is written for CTA pairs");
   if (lane == 0) {
     for (int s = 0; s < D; ++s) mbar_init(bars + 8 * s, 1);
-    if (!FLAT && warp == 0)
+    if (warp == 0)
       for (int i = 0; i < 2; ++i) {
         mbar_init(rbar + 8 * i, 1);
         mbar_init(fbar + 8 * i, 1);
@@ -456,7 +417,7 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
     fence_mbar_init();
   }
   __syncwarp();
-  if constexpr (!FLAT) cluster_arrive();       // the partner may use this CTA's barriers after its wait
+  cluster_arrive();                            // the partner may use this CTA's barriers after its wait
   uint32_t cs = 0, phase = 0;                  // ring position of the next stage to consume
   uint32_t in_flight = 0;                      // lane 0: stages issued and not consumed
   bool ok = true;
@@ -626,9 +587,7 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
     if (has0) put_tile<NTT>(wslots + (warp * 2 + 0) * TILEF + lane * 4 * NTT, p0);
     if (has1) put_tile<NTT>(wslots + (warp * 2 + 1) * TILEF + lane * 4 * NTT, acc);
     __syncthreads();
-    if constexpr (!FLAT) {
-      if (pass == 0) cluster_wait();          // the partner's barriers are initialised
-    }
+    if (pass == 0) cluster_wait();            // the partner's barriers are initialised
     if (FL > 0) {
       const uint32_t t_lo = F0 / G, t_hi = (F1 - 1) / G;
       const uint32_t par = pass & 1u, use = (pass >> 1) & 1u;
@@ -656,30 +615,6 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
         }
         if (whole) {
           if (any) store_tile<TILES, NT8>(y, s, tt, m0, M, N, lane);
-        } else if constexpr (FLAT) {
-          // Cut by a CTA boundary: CTAs cf .. cl meet this tile.  Store this
-          // CTA's partial, take a ticket; the last ticket adds all slots in
-          // CTA order, writes Y and clears the counter.  Every CTA takes part
-          // even after a timeout, so the counters always return to zero.
-          const uint32_t T = ntiles * G, Cn = gridDim.x;
-          const uint32_t cf = flat_owner(tb, T, Cn), cl = flat_owner(te - 1, T, Cn);
-          put_tile<NTT>(ws_slots + (size_t)(2 * blockIdx.x + (tt == t_lo ? 0u : 1u)) * TILEF + lane * 4 * NTT, s);
-          __threadfence();
-          __syncwarp();
-          uint32_t ticket = 0;
-          if (lane == 0) ticket = atomicAdd(ws_cnt + tt, 1u);
-          ticket = __shfl_sync(0xFFFFFFFFu, ticket, 0);
-          if (ticket == cl - cf) {
-            __threadfence();
-            float r[NTT][4];
-            zero_tile<NTT>(r);
-            for (uint32_t c2 = cf; c2 <= cl; ++c2) {
-              const uint32_t first2 = flat_start(T, c2, Cn) / G;
-              add_tile_l2<NTT>(r, ws_slots + (size_t)(2 * c2 + (tt == first2 ? 0u : 1u)) * TILEF + lane * 4 * NTT);
-            }
-            store_tile<TILES, NT8>(y, r, tt, m0, M, N, lane);
-            if (lane == 0) ws_cnt[tt] = 0u;
-          }
         } else if (te > F1) {
           // Rank 0's last tile continues in rank 1: push the partial there.
           if (pass >= 2 && !mbar_wait_cluster(fbar + 8 * par, use ^ 1u)) { ok = false; continue; }

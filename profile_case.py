@@ -64,14 +64,14 @@ def main():
         else:
             packed = [nvq.int4_pack_weights(codes, scales, a.N, a.K) for _ in range(a.copies)]
         y = torch.empty(a.M, a.N, dtype=torch.bfloat16, device=dev)
-        ws = torch.zeros(max(16, nvq.w4a16_workspace_bytes(a.M, a.N, a.K)), dtype=torch.uint8, device=dev)
+        ws = torch.empty(max(16, nvq.w4a16_workspace_bytes(a.M, a.N, a.K)), dtype=torch.uint8, device=dev)
         calls = [0]
 
         def run():
             pc, ps = packed[calls[0] % len(packed)]
             calls[0] += 1
             if a.sparse:
-                nvq.w4a16_sparse24_gemm(x, pc, ps, a.N, y=y, workspace=ws)
+                nvq.w4a16_sparse24_gemm(x, pc, ps, a.N, y=y)
             else:
                 nvq.w4a16_gemm(x, pc, ps, a.N, y=y, workspace=ws)
         wbytes = a.N * a.K * 3 / 8 if a.sparse else a.N * a.K / 2
@@ -153,13 +153,12 @@ def crossover(a, dev):
         xs = torch.empty(max(1, nvq.nvfp4_scales_bytes(M, K)), dtype=torch.uint8, device=dev)
         tx = torch.empty(1, dtype=torch.float32, device=dev)
         ws = torch.empty(max(16, nvq.nvfp4_quantize_workspace_bytes(M, K)), dtype=torch.uint8, device=dev)
-        dws = torch.zeros(max(16, nvq.w4a16_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
         k = [0]
 
         def w4a16():
             pc, ps = packed[k[0] % copies]
             k[0] += 1
-            nvq.w4a16_gemm(x, pc, ps, N, y=y, workspace=dws)
+            nvq.w4a16_gemm(x, pc, ps, N, y=y)
 
         def w4a4():
             wk = fp4[k[0] % copies]

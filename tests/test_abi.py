@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.nvq_abi_version() == 2
+    assert L.nvq_abi_version() == 1
     for code, name in nvq.STATUS.items():
         assert L.nvq_status_string(code).decode() == name
 
@@ -41,15 +41,8 @@ def test_size_helpers(L):
     assert L.nvfp4_scales_bytes(10, 100) == 0          # K % 64 != 0
     assert L.nvfp4_quantize_workspace_bytes(0, 64) == 0
     assert L.nvfp4_quantize_workspace_bytes(128, 512) > 0
-    # M <= 32: one ticket per 32-row tile (256-aligned), then two partial tiles
-    # of 32 rows x 8 NT8 columns (fp32) per CTA, for up to 2 CTAs per SM (148
-    # SMs when no GPU is visible)
-    sms = 148
-    assert L.w4a16_workspace_bytes(1, 4096, 4096) == 512 + 2 * 2 * sms * 256 * 4
-    assert L.w4a16_workspace_bytes(8, 4096, 128) == 512 + 2 * 2 * sms * 256 * 4
-    assert L.w4a16_workspace_bytes(16, 256, 4096) == 256 + 2 * 2 * sms * 512 * 4
-    assert L.w4a16_workspace_bytes(32, 24576, 4096) == 3072 + 2 * 2 * sms * 1024 * 4
-    assert L.w4a16_workspace_bytes(33, 4096, 4096) == 0               # several batch tiles: no workspace
+    assert L.w4a16_workspace_bytes(1, 4096, 4096) == 0          # partial sums stay on chip
+    assert L.w4a16_workspace_bytes(4, 256, 4096) == 0
     assert L.w4a16_workspace_bytes(4096, 4096, 4096) == 0
 
 
@@ -69,13 +62,9 @@ def test_scale_offset_map_matches_the_oracles_layout(L):
 def test_workspace_bytes_by_operation(L):
     assert L.nvq_workspace_bytes(0, 8192, 0, 4096) == L.nvfp4_quantize_workspace_bytes(8192, 4096) > 0
     assert L.nvq_workspace_bytes(1, 8192, 4096, 4096) == 0
-    assert L.nvq_workspace_bytes(2, 16, 4096, 4096) == L.w4a16_workspace_bytes(16, 4096, 4096) > 0
+    assert L.nvq_workspace_bytes(2, 16, 4096, 4096) == L.w4a16_workspace_bytes(16, 4096, 4096) == 0
     assert L.nvq_workspace_bytes(3, 4096, 24576, 4096) == L.nvq_linear_workspace_bytes(4096, 24576, 4096, -1) > 0
-    # nvq_linear: the decode region (sized for M = 32) first, then the W4A4 outputs
-    dec = L.w4a16_workspace_bytes(32, 24576, 4096)
-    dec = (dec + 255) // 256 * 256
-    assert L.nvq_workspace_bytes(3, 1, 24576, 4096) == dec
-    assert L.nvq_linear_workspace_bytes(4096, 24576, 4096, -1) > dec
+    assert L.nvq_workspace_bytes(3, 1, 24576, 4096) == 0
     assert L.nvq_workspace_bytes(7, 1, 1, 64) == 2 ** 64 - 1
 
 
@@ -131,10 +120,6 @@ def test_int4_calls_reject_bad_arguments(L):
     assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 48, 128, None, 0, None) == 2     # N % 32
     assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(ODD), 4, 256, 4096, None, 0, None) == 3    # y misaligned
     assert w(_vp(FAKE), _vp(FAKE), None, _vp(FAKE), 4, 256, 4096, None, 0, None) == 1         # NULL scales
-    need = L.w4a16_workspace_bytes(4, 256, 4096)
-    assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 256, 4096, None, 0, None) == 4    # no workspace
-    assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 256, 4096, _vp(FAKE), need - 1, None) == 4
-    assert w(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 256, 4096, _vp(ODD), need, None) == 3
 
 
 def test_row_shard_calls_reject_bad_arguments(L):
@@ -184,11 +169,10 @@ def test_phase_dispatch_host_rules(L):
     """nvq_linear: path choice by M, workspace sizing and argument checks (no GPU)."""
     c = L.nvq_default_crossover_m()
     assert c >= 1
-    dec = L.nvq_linear_workspace_bytes(c, 24576, 4096, -1)                     # W4A16 side: decode region only
-    assert dec >= L.w4a16_workspace_bytes(32, 24576, 4096) and dec % 256 == 0
+    assert L.nvq_linear_workspace_bytes(c, 24576, 4096, -1) == 0               # W4A16 side: no scratch
     big = L.nvq_linear_workspace_bytes(c + 1, 24576, 4096, -1)
-    assert big >= dec + (c + 1) * 4096 // 2 + L.nvfp4_scales_bytes(c + 1, 4096)   # + codes + scales at least
-    assert L.nvq_linear_workspace_bytes(64, 24576, 4096, 128) == dec            # caller's crossover wins
+    assert big >= (c + 1) * 4096 // 2 + L.nvfp4_scales_bytes(c + 1, 4096)       # codes + scales at least
+    assert L.nvq_linear_workspace_bytes(64, 24576, 4096, 128) == 0              # caller's crossover wins
     f = L.nvq_linear
     # W4A16 side without the packed weights / W4A4 side without the NVFP4 weights
     assert f(_vp(FAKE), 1, 256, 4096, _vp(FAKE), _vp(FAKE), _vp(FAKE), None, None, -1,
@@ -202,11 +186,9 @@ def test_phase_dispatch_host_rules(L):
              _vp(FAKE), _vp(ODD), 1 << 30, None) == 3
     assert f(_vp(FAKE), 4096, 256, 4100, _vp(FAKE), _vp(FAKE), _vp(FAKE), None, None, -1,
              _vp(FAKE), _vp(FAKE), 1 << 30, None) == 2
-    # W4A16 side keeps its own shape rules (N % 32) and needs its workspace region
+    # W4A16 side keeps its own shape rules (N % 32)
     assert f(_vp(FAKE), 1, 48, 4096, None, None, None, _vp(FAKE), _vp(FAKE), -1,
              _vp(FAKE), None, 0, None) == 2
-    assert f(_vp(FAKE), 1, 256, 4096, None, None, None, _vp(FAKE), _vp(FAKE), -1,
-             _vp(FAKE), None, 0, None) == 4
 
 
 def test_prefill_streamed_host_rules(L):
@@ -254,8 +236,8 @@ def test_sparse24_host_rules(L):
     assert p(_vp(FAKE), None, _vp(FAKE), 32, 128, _vp(FAKE), _vp(FAKE), None) == 1
     assert p(_vp(FAKE), _vp(FAKE), _vp(FAKE), 32, 128, _vp(ODD), _vp(FAKE), None) == 3
     g = L.w4a16_sparse24_gemm
-    assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 24, 128, None, 0, None) == 2
-    assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 48, 128, None, 0, None) == 2
-    assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(ODD), 4, 256, 4096, None, 0, None) == 3
-    assert g(_vp(FAKE), None, _vp(FAKE), _vp(FAKE), 4, 256, 4096, None, 0, None) == 1
-    assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 0, 256, 4096, None, 0, None) == 0
+    assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 24, 128, None) == 2
+    assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 4, 48, 128, None) == 2
+    assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(ODD), 4, 256, 4096, None) == 3
+    assert g(_vp(FAKE), None, _vp(FAKE), _vp(FAKE), 4, 256, 4096, None) == 1
+    assert g(_vp(FAKE), _vp(FAKE), _vp(FAKE), _vp(FAKE), 0, 256, 4096, None) == 0

@@ -67,87 +67,3 @@ def test_every_tile_written_once(G):
             got = producers(ntiles, G, nclu)
             assert sorted(got) == list(range(ntiles))
             assert all(len(v) == 1 for v in got.values()), (ntiles, G, nclu)
-
-
-# ------------------------------------------------------------------ even split over the whole grid (M <= 32)
-
-def flat_start(T, c, C):
-    return (T * c) // C
-
-
-def flat_owner(u, T, C):
-    return ((u + 1) * C - 1) // T
-
-
-def flat_producers(ntiles, G, C):
-    """Who writes each tile under the even split: a warp that covered it whole,
-    the CTA that holds it whole (its warps' partials summed), or the CTA that
-    draws the last ticket of a tile cut by CTA boundaries (partials from the
-    slots of CTAs cf..cl).  Also checks that every contributor stores into a
-    slot that no other (CTA, tile) uses and that the reader finds it there."""
-    T = ntiles * G
-    out, tickets, slots = {}, {}, {}
-    for c in range(C):
-        F0, F1 = flat_start(T, c, C), flat_start(T, c + 1, C)
-        FL = F1 - F0
-        assert FL >= 1                                       # the host never launches more CTAs than units
-        for warp in range(W):
-            f0, f1 = F0 + split_at(FL, warp, 3), F0 + split_at(FL, warp + 1, 3)
-            if f1 <= f0:
-                continue
-            wt_first, g_first = divmod(f0, G)
-            nt, g, left = wt_first, g_first, f1 - f0
-            while left > 0:
-                n = min(left, SG, G - g)
-                g, left = g + n, left - n
-                if g == G:
-                    if not (nt == wt_first and g_first != 0):
-                        out.setdefault(nt, []).append(("warp", c, warp))
-                    g, nt = 0, nt + 1
-        t_lo, t_hi = F0 // G, (F1 - 1) // G
-        for tt in range(t_lo, t_hi + 1):
-            tb, te = tt * G, tt * G + G
-            takers = [w2 for w2 in range(W)
-                      if (lambda a, b: a < b and a < te and b > tb and not (a <= tb and b >= te))(
-                          F0 + split_at(FL, w2, 3), F0 + split_at(FL, w2 + 1, 3))]
-            if tb >= F0 and te <= F1:
-                if takers:
-                    out.setdefault(tt, []).append(("cta", c))
-                continue
-            assert takers                                    # a cut tile always has a partial here
-            cf, cl = flat_owner(tb, T, C), flat_owner(te - 1, T, C)
-            assert cf <= c <= cl and cl > cf
-            slot = 2 * c + (0 if tt == t_lo else 1)
-            assert slot not in slots
-            slots[slot] = (c, tt)
-            tickets.setdefault(tt, []).append(c)
-            if len(tickets[tt]) == cl - cf + 1:              # whichever CTA comes last: same reader
-                read = [2 * c2 + (0 if tt == flat_start(T, c2, C) // G else 1) for c2 in range(cf, cl + 1)]
-                assert [slots[r] for r in read] == [(c2, tt) for c2 in range(cf, cl + 1)]
-                out.setdefault(tt, []).append(("last", tt))
-    for tt, cs in tickets.items():
-        cf, cl = flat_owner(tt * G, T, C), flat_owner(tt * G + G - 1, T, C)
-        assert sorted(cs) == list(range(cf, cl + 1))
-    return out
-
-
-@pytest.mark.parametrize("G", [1, 2, 3, 5, 32, 96, 200])
-def test_even_split_writes_every_tile_once(G):
-    for ntiles in list(range(1, 20)) + [96, 128, 192, 768]:
-        T = ntiles * G
-        for C in (1, 2, 3, 7, 148, 296):
-            C = min(C, T)
-            got = flat_producers(ntiles, G, C)
-            assert sorted(got) == list(range(ntiles)), (ntiles, G, C)
-            assert all(len(v) == 1 for v in got.values()), (ntiles, G, C)
-
-
-def test_flat_owner_inverts_flat_start():
-    for T in (1, 5, 32, 4096, 24576, 393216):
-        for C in (1, 3, 148, 296):
-            if C > T:
-                continue
-            for c in range(C):
-                a, b = flat_start(T, c, C), flat_start(T, c + 1, C)
-                for u in {a, b - 1, (a + b) // 2}:
-                    assert flat_owner(u, T, C) == c

@@ -330,27 +330,6 @@ def test_w4a16_qwen3_8b_decode_full_size(layer):
         assert ok, (name, M, worst)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (8, 288, 384), (16, 6144, 1024), (32, 1024, 12288),
-                                   (5, 32, 128)])
-def test_w4a16_workspace_tickets_return_to_zero_and_calls_repeat(M, N, K):
-    """The even split finishes tiles cut by CTA boundaries through the
-    workspace; after every call its tile counters are zero again, so the same
-    workspace serves the next call, which gives the same bits."""
-    x = synth.activations(M, K, seed=M * 31 + N)
-    w = synth.weights(N, K, seed=K + 9)
-    packed = gpu_int4(w)
-    ws = torch.zeros(nvq.w4a16_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
-    xg = x.cuda()
-    y1 = nvq.w4a16_gemm(xg, packed[2], packed[3], N, workspace=ws)
-    y2 = nvq.w4a16_gemm(xg, packed[2], packed[3], N, workspace=ws)
-    nvq.check_device_error()
-    assert not ws[: (N // 32) * 4].any()
-    assert torch.equal(y1, y2)
-    u, s_bits = oracle_int4(w)
-    ok, worst = onv.within_tolerance(bf16_to_f64(y1), oint4.w4a16_ref(bf16_to_f64(x), oint4.dequantize(u, s_bits)))
-    assert ok, (M, N, K, worst)
-
-
 @pytest.mark.parametrize("M", synth.CROSSOVER_BATCHES)
 def test_crossover_sweep_both_paths_sampled(M):
     """gate_up (K=4096, N=24576): one master W quantized both ways, both paths at M."""
