@@ -59,8 +59,8 @@ template <int NT8, bool SPARSE = false>
 struct Cfg {
   using U = Unit<SPARSE>;
   static constexpr int W = 8;                          // warps per CTA (two CTAs per SM)
-  static constexpr int SG = 2;                         // units per ring stage
-  static constexpr int D = NT8 == 1 ? 3 : 6;           // ring stages per warp
+  static constexpr int SG = 3;                         // units per ring stage
+  static constexpr int D = NT8 == 1 ? 2 : 4;           // ring stages per warp
   static constexpr int THREADS = W * 32;
   static constexpr int MIN_CTAS = NT8 == 1 ? 2 : 1;     // CTAs per SM the register budget must allow
   static constexpr int STAGE = SG * U::BYTES;           // codes first, then the scales
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
       for (int t = 0; t < NT8; ++t)
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          xa[t][v] = (!SPARSE && C::XDB && live[t]) ? __ldg(xrow[t] + g_first * 16u + v) : make_uint4(0, 0, 0, 0);
+          xa[t][v] = (!SPARSE && C::XDB) ? __ldg(xrow[t] + g_first * 16u + v) : make_uint4(0, 0, 0, 0);
           xb[t][v] = make_uint4(0, 0, 0, 0);
         }
       uint32_t nt = wt_first, g = g_first, left = nf;
@@ -511,14 +511,14 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
               for (int t = 0; t < NT8; ++t)
 #pragma unroll
                 for (int v = 0; v < 4; ++v)
-                  if (live[t]) nxt[t][v] = __ldg(xrow[t] + gn * 16u + v);
+                  nxt[t][v] = __ldg(xrow[t] + gn * 16u + v);      // rows >= M read row 0 (discarded)
               dense_unit<NT8, C::ONES>(stage + i * UC + lane * 16, cur, d);
             } else {
 #pragma unroll
               for (int t = 0; t < NT8; ++t)
 #pragma unroll
                 for (int v = 0; v < 4; ++v)
-                  if (live[t]) xa[t][v] = __ldg(xrow[t] + (g + i) * 16u + v);
+                  xa[t][v] = __ldg(xrow[t] + (g + i) * 16u + v);
               dense_unit<NT8, C::ONES>(stage + i * UC + lane * 16, xa, d);
             }
             // Scale word tt of this lane: rows 16 tt + g (low half) and 16 tt + g + 8 (high half).
