@@ -40,9 +40,11 @@
 namespace nvq {
 namespace w4a4 {
 
-constexpr int BM = 128, BN = 256;            // rows of A per CTA, columns of one MMA / output tile
+constexpr int BM = 128, BN = 256;
 constexpr int BKB = 128;                      // k-stage width in bytes (256 FP4 elements)
+constexpr int STAGES = 3;
 constexpr int A_BYTES = BM * BKB;             // 16 KB
+constexpr int B_BYTES = BN * BKB;             // 32 KB
 constexpr int SFA_BYTES = 4 * 512;            // 4 k-atoms of the 128 A rows
 constexpr int SFB_BYTES = 2 * 4 * 512;        // 2 row-atoms x 4 k-atoms of the 256 B rows
 constexpr int EPI_WARPS = 8;
@@ -54,35 +56,23 @@ constexpr uint32_t ACC1_COL = 128;            // accumulator 1 starts here (over
 constexpr uint32_t SF_COL0 = 384;
 constexpr uint32_t SF_SLOT_COLS = 48;         // one k-stage: 4 x (4 A + 8 B) columns
 constexpr uint32_t SF_SLOTS = 2;
+
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
+constexpr int OFF_SFA = OFF_C + EPI_WARPS * C_BYTES;
+constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+// full[S], empty[S], acc_full[2], acc_empty[2], overlap_free, sf_full[2], drain, scales_in[S]
+constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 1 + SF_SLOTS + 1 + STAGES;
+constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
+constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;    // + slack for 1024-byte alignment
+static_assert(SMEM_BYTES <= 232448, "smem budget");
 static_assert(SF_COL0 + SF_SLOTS * SF_SLOT_COLS <= TMEM_COLS && ACC1_COL + BN <= SF_COL0, "TMEM budget");
 
-// Shared-memory layout.  One CTA (PAIR = false): a 128 x 256 output tile, B's
-// 256 rows loaded by the CTA.  CTA pair (PAIR = true): a 256 x 256 tile, each
-// CTA loads its 128 rows of A and 128 of the 256 rows of B, and one MMA
-// instruction from the pair leader drives both CTAs' tensor cores, so each
-// CTA stages a third less operand data per FLOP and more k-stages fit.
-template <bool PAIR>
-struct Geo {
-  static constexpr int STAGES = PAIR ? 4 : 3;
-  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // rows of B this CTA loads per k-stage
-  static constexpr int B_BYTES = B_ROWS * BKB;
-  static constexpr int TILE_M = PAIR ? 2 * BM : BM;  // rows of one output tile
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_SFA = OFF_C + EPI_WARPS * C_BYTES;
-  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-  static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
-  // full[S], empty[S], acc_full[2], acc_empty[2], overlap_free, sf_full[2], drain, scales_in[S]
-  static constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 1 + SF_SLOTS + 1 + STAGES;
-  static constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;    // + slack for 1024-byte alignment
-  static_assert(SMEM_BYTES <= 232448, "smem budget");
-  // Instruction descriptor, kind::mxf4nvf4: A/B E2M1 (format 1), K-major,
-  // UE4M3 scales, N >> 3 in bits 17..22, M >> 4 in bits 24..28 (M = 256 for a pair).
-  static constexpr uint32_t IDESC =
-      (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(TILE_M >> 4) << 24);
-};
+// Instruction descriptor, kind::mxf4nvf4: A/B E2M1 (format 1), K-major,
+// UE4M3 scales, N >> 3 in bits 17..22, M >> 4 in bits 24..28.
+constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
 struct Params {
   const uint8_t* x_scales;
@@ -93,7 +83,6 @@ struct Params {
   uint32_t num_m_tiles, num_n_tiles, num_k_stages;
   uint32_t k_atoms;        // K / 64: scale atoms per 128-row tile
   uint32_t n_row_atoms;    // padded N / 128
-  uint32_t m_row_atoms;    // padded M / 128: 128-row atoms of A's (and H's) tiled scales
   uint32_t m_fastest;      // 1: tile index runs over row blocks first (A re-read per wave)
   // SiLU * mul epilogue only (B rows interleaved in blocks of 128: gate, up, gate, up, ...)
   uint8_t* h_codes;        // [M, N/2 / 2] E2M1 codes of H = silu(gate) * up
@@ -210,21 +199,15 @@ __device__ __forceinline__ uint32_t acc_col(uint32_t buf) { return buf ? ACC1_CO
 
 // EPI 0: Y = BF16(alpha acc).  EPI 1: B rows interleaved in blocks of 128 (gate,
 // up, gate, up, ...); H = silu(gate) * up quantized to NVFP4 with a static t_h.
-// PAIR: launched in clusters of two CTAs that share each 256 x 256 tile; the
-// pair leader (cluster rank 0) issues the MMAs for both, every barrier the MMA
-// thread waits on lives in the leader and counts both CTAs' arrivals, and the
-// leader's commits arrive in both CTAs.
-template <int EPI, bool PAIR>
+template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                   const __grid_constant__ CUtensorMap tmap_y, const Params p) {
-  using GEO = Geo<PAIR>;
-  constexpr int STAGES = GEO::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
-  const uint32_t bar_full = sbase + GEO::OFF_BAR;             // + 8 s
+  const uint32_t bar_full = sbase + OFF_BAR;                  // + 8 s
   const uint32_t bar_empty = bar_full + 8 * STAGES;           // + 8 s
   const uint32_t bar_acc_full = bar_empty + 8 * STAGES;       // + 8 b
   const uint32_t bar_acc_empty = bar_acc_full + 16;           // + 8 b
@@ -232,14 +215,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
   const uint32_t bar_sf_full = bar_overlap + 8;               // + 8 slot
   const uint32_t bar_drain = bar_sf_full + 8 * SF_SLOTS;
   const uint32_t bar_sc_in = bar_drain + 8;                   // + 8 s: the stage's scale atoms landed
-  uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(smem + GEO::OFF_TMEM_PTR);
-  const uint32_t rank = PAIR ? cluster_rank() : 0u;           // this CTA's half of a pair tile
-  const bool leader = rank == 0u;
-  const uint32_t unit = PAIR ? (blockIdx.x >> 1) : blockIdx.x;          // tiles are walked per pair
-  const uint32_t nunits = PAIR ? (gridDim.x >> 1) : gridDim.x;
-  // The leader's copy of a barrier, as a shared::cluster address (this CTA's own when not paired).
-  auto lead = [&](uint32_t bar) -> uint32_t { return PAIR ? map_to_rank(bar, 0) : bar; };
-  constexpr uint32_t kSides = PAIR ? 2u : 1u;
+  uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(smem + OFF_TMEM_PTR);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -249,11 +225,11 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_acc_full + 8 * b, 1);
-      mbar_init(bar_acc_empty + 8 * b, EPI_WARPS * kSides);   // one arrive per epilogue warp (of both CTAs)
+      mbar_init(bar_acc_empty + 8 * b, EPI_WARPS);            // one arrive per epilogue warp
     }
-    mbar_init(bar_overlap, EPI_WARPS * kSides);
+    mbar_init(bar_overlap, EPI_WARPS);
     for (uint32_t k = 0; k < SF_SLOTS; ++k) {
-      mbar_init(bar_sf_full + 8 * k, 4 * kSides);             // one arrive per scale-writer warp
+      mbar_init(bar_sf_full + 8 * k, 4);                      // one arrive per scale-writer warp
     }
     mbar_init(bar_drain, 1);
     fence_mbar_init();
@@ -262,20 +238,11 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     if (EPI == 0) prefetch_tensormap(&tmap_y);
   }
   if (warp == 0) {
-    if constexpr (PAIR) {
-      tmem_alloc_pair(smem_addr(tmem_ptr_smem), TMEM_COLS);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(smem_addr(tmem_ptr_smem), TMEM_COLS);
-      tmem_relinquish();
-    }
+    tmem_alloc(smem_addr(tmem_ptr_smem), TMEM_COLS);
+    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
-  if constexpr (PAIR) {                       // both CTAs' barriers and TMEM are ready before any cross-CTA use
-    cluster_arrive();
-    cluster_wait();
-  }
   tc_fence_after();
   const uint32_t tmem_base = *tmem_ptr_smem;
   const uint32_t num_tiles = p.num_m_tiles * p.num_n_tiles;
@@ -287,116 +254,82 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       uint32_t stage = 0, phase = 0;
       uint32_t pending = 0, pending_parity = 0;               // per-stage bit masks
       bool ok = true;
-      for (uint32_t tile = unit; tile < num_tiles && ok; tile += nunits) {
+      for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         uint32_t mt, nt;
         tile_coords(tile, p, mt, nt);
-        const uint32_t a_row = mt * GEO::TILE_M + rank * BM;   // first row of A (and of Y) of this CTA
-        const uint32_t b_row = nt * BN + rank * (BN - GEO::B_ROWS);
         const uint32_t nb_atoms = min(2u, p.n_row_atoms - 2 * nt);
         for (uint32_t ks = 0; ks < p.num_k_stages; ++ks) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1)) { ok = false; break; }
           const uint32_t natoms = min(4u, p.k_atoms - 4 * ks);
           // The scale atoms complete on a barrier of their own and go first, so
           // the scale writers can move them into TMEM while the operands land.
-          // Each CTA loads the scales of its own A rows and of all 256 B rows.
           const uint32_t sb = bar_sc_in + 8 * stage;
           mbar_arrive_expect_tx(sb, natoms * 512u * (1u + nb_atoms));
-          // A pair tile may reach past A's last 128-row atom (M <= 128 rows below
-          // it): that CTA's rows are all padding, their products never stored,
-          // so it reads the last atom instead of past the end of the buffer.
-          const uint32_t a_atom = min(a_row / BM, p.m_row_atoms - 1u);
-          bulk_load(sbase + GEO::OFF_SFA + stage * SFA_BYTES,
-                    p.x_scales + ((size_t)a_atom * p.k_atoms + 4 * ks) * 512u, natoms * 512u, sb);
+          bulk_load(sbase + OFF_SFA + stage * SFA_BYTES,
+                    p.x_scales + ((size_t)mt * p.k_atoms + 4 * ks) * 512u, natoms * 512u, sb);
           for (uint32_t a = 0; a < nb_atoms; ++a)
-            bulk_load(sbase + GEO::OFF_SFB + stage * SFB_BYTES + a * 2048u,
+            bulk_load(sbase + OFF_SFB + stage * SFB_BYTES + a * 2048u,
                       p.w_scales + ((size_t)(2 * nt + a) * p.k_atoms + 4 * ks) * 512u, natoms * 512u, sb);
           const uint32_t fb = bar_full + 8 * stage;
-          if constexpr (PAIR) {
-            // Both CTAs' operand bytes count toward the leader's full barrier.
-            const uint32_t lfb = lead(fb);
-            if (leader) mbar_arrive_expect_tx(fb, 2 * (A_BYTES + GEO::B_BYTES));
-            tma_load_2d_pair(sbase + GEO::OFF_A + stage * A_BYTES, &tmap_a, lfb, (int)(ks * BKB), (int)a_row, pol);
-            tma_load_2d_pair(sbase + GEO::OFF_B + stage * GEO::B_BYTES, &tmap_b, lfb, (int)(ks * BKB), (int)b_row,
-                             pol);
-          } else {
-            mbar_arrive_expect_tx(fb, A_BYTES + GEO::B_BYTES);
-            tma_load_2d(sbase + GEO::OFF_A + stage * A_BYTES, &tmap_a, fb, (int)(ks * BKB), (int)a_row, pol);
-            tma_load_2d(sbase + GEO::OFF_B + stage * GEO::B_BYTES, &tmap_b, fb, (int)(ks * BKB), (int)b_row, pol);
-          }
+          mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+          tma_load_2d(sbase + OFF_A + stage * A_BYTES, &tmap_a, fb, (int)(ks * BKB), (int)(mt * BM), pol);
+          tma_load_2d(sbase + OFF_B + stage * B_BYTES, &tmap_b, fb, (int)(ks * BKB), (int)(nt * BN), pol);
           pending |= 1u << stage;
           pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
-      // Let every copy issued into shared memory land before the CTA exits (a
-      // pair's operand copies complete on the leader's barriers: the leader
-      // waits for both CTAs' bytes, and the cluster barrier below keeps the
-      // other CTA alive meanwhile).
+      // Let every copy issued into shared memory land before the CTA exits.
       for (int s2 = 0; s2 < STAGES; ++s2)
         if (pending & (1u << s2)) {
           mbar_wait_drain(bar_sc_in + 8 * s2, (pending_parity >> s2) & 1u, 200000000ull);
-          if (leader) mbar_wait_drain(bar_full + 8 * s2, (pending_parity >> s2) & 1u, 200000000ull);
+          mbar_wait_drain(bar_full + 8 * s2, (pending_parity >> s2) & 1u, 200000000ull);
         }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (the pair leader only)
-    if (leader) {
-      const uint64_t adesc0 = smem_desc(sbase + GEO::OFF_A, 0, 1024, kSwizzle128B);
-      const uint64_t bdesc0 = smem_desc(sbase + GEO::OFF_B, 0, 1024, kSwizzle128B);
-      uint32_t stage = 0, phase = 0, acc_par = 0, local = 0;
-      uint32_t slot = 0, slot_phase = 0;
-      bool ok = true;
-      auto wait = [&](uint32_t bar, uint32_t par) {
-        return PAIR ? warp_mbar_wait_cluster(bar, par) : warp_mbar_wait(bar, par);
-      };
-      for (uint32_t tile = unit; tile < num_tiles && ok; tile += nunits, ++local) {
-        const uint32_t buf = local & 1u;
-        // This accumulator was drained (tile - 2), and the columns it shares with
-        // the other accumulator were read for the previous tile.
-        if (!(ok = wait(bar_acc_empty + 8 * buf, ((acc_par >> buf) & 1u) ^ 1u))) break;
-        acc_par ^= 1u << buf;
-        if (local > 0 && !(ok = wait(bar_overlap, (local - 1) & 1u))) break;
+    // ------------------------------------------------------------ MMA issuer
+    const uint64_t adesc0 = smem_desc(sbase + OFF_A, 0, 1024, kSwizzle128B);
+    const uint64_t bdesc0 = smem_desc(sbase + OFF_B, 0, 1024, kSwizzle128B);
+    uint32_t stage = 0, phase = 0, acc_par = 0, local = 0;
+    uint32_t slot = 0, slot_phase = 0;
+    bool ok = true;
+    for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+      const uint32_t buf = local & 1u;
+      // This accumulator was drained (tile - 2), and the columns it shares with
+      // the other accumulator were read for the previous tile.
+      if (!(ok = warp_mbar_wait(bar_acc_empty + 8 * buf, ((acc_par >> buf) & 1u) ^ 1u))) break;
+      acc_par ^= 1u << buf;
+      if (local > 0 && !(ok = warp_mbar_wait(bar_overlap, (local - 1) & 1u))) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc_col(buf);
+      for (uint32_t ks = 0; ks < p.num_k_stages; ++ks) {
+        if (!(ok = warp_mbar_wait(bar_full + 8 * stage, phase))) break;
+        if (!(ok = warp_mbar_wait(bar_sf_full + 8 * slot, slot_phase))) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc_col(buf);
-        for (uint32_t ks = 0; ks < p.num_k_stages; ++ks) {
-          if (!(ok = wait(bar_full + 8 * stage, phase))) break;
-          if (!(ok = wait(bar_sf_full + 8 * slot, slot_phase))) break;
-          tc_fence_after();
-          if (lane == 0) {
-            const uint64_t ad = adesc0 + stage * (A_BYTES >> 4);
-            const uint64_t bd = bdesc0 + stage * (GEO::B_BYTES >> 4);
-            const uint32_t sf = tmem_base + SF_COL0 + SF_SLOT_COLS * slot;
-            const uint32_t natoms = min(4u, p.k_atoms - 4 * ks);
-            for (uint32_t j = 0; j < natoms; ++j) {   // 32 bytes (64 FP4 elements) per k step
-              if constexpr (PAIR)
-                tc_mma_nvf4_pair(d_tmem, ad + 2 * j, bd + 2 * j, GEO::IDESC, sf + 4 * j, sf + 16 + 8 * j, (ks | j) != 0u);
-              else
-                tc_mma_nvf4(d_tmem, ad + 2 * j, bd + 2 * j, GEO::IDESC, sf + 4 * j, sf + 16 + 8 * j, (ks | j) != 0u);
-            }
-            // Frees this stage's operands (in both CTAs) and, two stages later, its scale slot.
-            if constexpr (PAIR) tc_commit_pair(bar_empty + 8 * stage, 0x3);
-            else tc_commit(bar_empty + 8 * stage);
-          }
-          __syncwarp();
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
-          if (++slot == SF_SLOTS) { slot = 0; slot_phase ^= 1; }
-        }
-        if (!ok) break;
         if (lane == 0) {
-          if constexpr (PAIR) tc_commit_pair(bar_acc_full + 8 * buf, 0x3);
-          else tc_commit(bar_acc_full + 8 * buf);
+          const uint64_t ad = adesc0 + stage * (A_BYTES >> 4);
+          const uint64_t bd = bdesc0 + stage * (B_BYTES >> 4);
+          const uint32_t sf = tmem_base + SF_COL0 + SF_SLOT_COLS * slot;
+          const uint32_t natoms = min(4u, p.k_atoms - 4 * ks);
+          for (uint32_t j = 0; j < natoms; ++j)     // 32 bytes (64 FP4 elements) per k step
+            tc_mma_nvf4(d_tmem, ad + 2 * j, bd + 2 * j, IDESC, sf + 4 * j, sf + 16 + 8 * j, (ks | j) != 0u);
+          tc_commit(bar_empty + 8 * stage);                    // also frees this stage's scale slot
         }
         __syncwarp();
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        if (++slot == SF_SLOTS) { slot = 0; slot_phase ^= 1; }
       }
-      // Every MMA this thread issued has finished before TMEM is released.
-      if (lane == 0) {
-        if constexpr (PAIR) tc_commit_pair(bar_drain, 0x1);
-        else tc_commit(bar_drain);
-        mbar_wait_drain(bar_drain, 0, 200000000ull);
-      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(bar_acc_full + 8 * buf);
       __syncwarp();
     }
+    // Every MMA this thread issued has finished before TMEM is released.
+    if (lane == 0) {
+      tc_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0, 200000000ull);
+    }
+    __syncwarp();
   } else if (warp >= 2 + EPI_WARPS) {
     // ------------------------------------------------------------ scale writers
     const uint32_t q = warp & 3u;                             // TMEM sub-partition of this warp
@@ -408,7 +341,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     // (a tcgen05.commit costs the MMA thread about as much as an MMA).
     uint32_t lag_stage = 0, lag_phase = 0, kg = 0;
     bool ok = true;
-    for (uint32_t tile = unit; tile < num_tiles && ok; tile += nunits) {
+    for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       for (uint32_t ks = 0; ks < p.num_k_stages; ++ks, ++kg) {
         if (kg >= SF_SLOTS) {
           if (!(ok = warp_mbar_wait(bar_empty + 8 * lag_stage, lag_phase))) break;
@@ -416,8 +349,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         }
         if (!(ok = warp_mbar_wait(bar_sc_in + 8 * stage, phase))) break;   // this stage's scale atoms
         tc_fence_after();
-        const uint8_t* sfa = smem + GEO::OFF_SFA + stage * SFA_BYTES + 16 * lane;
-        const uint8_t* sfb = smem + GEO::OFF_SFB + stage * SFB_BYTES + 16 * lane;
+        const uint8_t* sfa = smem + OFF_SFA + stage * SFA_BYTES + 16 * lane;
+        const uint8_t* sfb = smem + OFF_SFB + stage * SFB_BYTES + 16 * lane;
         const uint32_t col = lane_base + tmem_base + SF_COL0 + SF_SLOT_COLS * slot;
         const uint32_t natoms = min(4u, p.k_atoms - 4 * ks);
         // Atom row `lane` holds rows lane, lane+32, lane+64, lane+96 (4 bytes each);
@@ -449,10 +382,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          if constexpr (PAIR) mbar_arrive_remote(lead(bar_sf_full + 8 * slot));
-          else mbar_arrive(bar_sf_full + 8 * slot);
-        }
+        if (lane == 0) mbar_arrive(bar_sf_full + 8 * slot);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
         if (++slot == SF_SLOTS) slot = 0;
       }
@@ -463,17 +393,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     const uint32_t h = (warp - 2) >> 2;                       // which 64-column chunk of each pair
     const uint32_t row = q * 32 + lane;                       // row of the tile held by this thread
     const float alpha = __ldg(p.t_x) * __ldg(p.t_w);
-    // Release the shared TMEM columns / the accumulator to the MMA thread (the leader's barriers).
-    auto release = [&](uint32_t bar) {
-      if constexpr (PAIR) mbar_arrive_remote(lead(bar));
-      else mbar_arrive(bar);
-    };
     if constexpr (EPI == 0) {
-    uint8_t* cbuf = smem + GEO::OFF_C + (warp - 2) * C_BYTES;   // this warp's 32 x 128 B staging
+    uint8_t* cbuf = smem + OFF_C + (warp - 2) * C_BYTES;      // this warp's 32 x 128 B staging
     const uint32_t cbuf_s = smem_addr(cbuf);
     uint32_t acc_par = 0, local = 0;
     bool dead = false;                                        // a wait ran out: skip work
-    for (uint32_t tile = unit; tile < num_tiles; tile += nunits, ++local) {
+    for (uint32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       uint32_t mt, nt;
       tile_coords(tile, p, mt, nt);
       const uint32_t buf = local & 1u;
@@ -490,7 +415,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) release(bar_overlap);
+      if (lane == 0) mbar_arrive(bar_overlap);
 #pragma unroll 1
       for (int part = 0; part < 2; ++part) {
         const uint32_t ch = part ? ch_second : ch_first;
@@ -514,14 +439,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         __syncwarp();
         const uint32_t col0 = nt * BN + ch * C_COLS;
         if (lane == 0 && col0 < p.N) {
-          tma_store_2d(&tmap_y, cbuf_s, (int)col0, (int)(mt * GEO::TILE_M + rank * BM + q * 32));
+          tma_store_2d(&tmap_y, cbuf_s, (int)col0, (int)(mt * BM + q * 32));
           bulk_commit();
         }
         if (part == 0) {
           tc_wait_ld();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) release(bar_acc_empty + 8 * buf);   // all of this tile's TMEM read
+          if (lane == 0) mbar_arrive(bar_acc_empty + 8 * buf);   // all of this tile's TMEM read
         }
       }
     }
@@ -532,7 +457,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       // SiLU * mul -> NVFP4.  Tile columns [0, 128) are gate rows of B, [128, 256)
       // the matching up rows; this warp owns H columns 64 h .. 64 h + 63 of the
       // tile (its gate chunk h and up chunk 2 + h) for rows 32 q .. 32 q + 31.
-      HTables& tb = *reinterpret_cast<HTables*>(smem + GEO::OFF_C);   // staging unused here
+      HTables& tb = *reinterpret_cast<HTables*>(smem + OFF_C);   // staging unused here
       const float t_h = __ldg(p.t_h);
       const uint32_t etid = threadIdx.x - 64u;                  // 0 .. 255 over the epilogue warps
       if (etid < 127u) build_h_table(tb, etid, t_h);
@@ -541,7 +466,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       const uint32_t hrow_bytes = p.N >> 2;                     // (N / 2) codes, two per byte
       uint32_t acc_par = 0, local = 0;
       bool dead = false;
-      for (uint32_t tile = unit; tile < num_tiles; tile += nunits, ++local) {
+      for (uint32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
         uint32_t mt, nt;
         tile_coords(tile, p, mt, nt);
         const uint32_t buf = local & 1u;
@@ -558,8 +483,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) release(bar_overlap);
-        const uint32_t grow = mt * GEO::TILE_M + rank * BM + row;
+        if (lane == 0) mbar_arrive(bar_overlap);
+        const uint32_t grow = mt * BM + row;
         uint32_t sword = 0;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {              // unrolled: vf is indexed at compile time
@@ -569,7 +494,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           if (part == 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) release(bar_acc_empty + 8 * buf);   // all of this tile's TMEM read
+            if (lane == 0) mbar_arrive(bar_acc_empty + 8 * buf);   // all of this tile's TMEM read
           }
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
@@ -591,21 +516,16 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         const uint32_t kb = (nt * 128u + h * 64u) >> 4;
         const size_t off = ((size_t)(grow >> 7) * p.h_katoms + (kb >> 2)) * 512u + (grow & 31u) * 16u +
                            ((grow & 127u) >> 5) * 4u;
-        if ((grow >> 7) < p.m_row_atoms) *reinterpret_cast<uint32_t*>(p.h_scales + off) = sword;   // padding rows: 0
+        *reinterpret_cast<uint32_t*>(p.h_scales + off) = sword;
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if constexpr (PAIR) {                       // the leader's MMAs into this CTA's TMEM have finished
-    cluster_arrive();
-    cluster_wait();
-  }
   if (warp == 0) {
     tc_fence_after();
-    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
-    else tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 

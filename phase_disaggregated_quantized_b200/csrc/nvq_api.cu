@@ -412,21 +412,17 @@ namespace {
 
 // EPI 0: y_bf16 receives Y.  EPI 1: h_* receive NVFP4(silu(gate) * up) with the
 // static scale t_h (B rows interleaved in blocks of 128: gate, up, ...).
-// PAIR: clusters of two CTAs share each 256 x 256 output tile (one MMA
-// instruction drives both SMs' tensor cores); otherwise one CTA per 128 x 256 tile.
-template <int EPI, bool PAIR>
+template <int EPI>
 nvq_status launch_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const float* t_x, const uint8_t* w_codes,
                        const uint8_t* w_scales, const float* t_w, void* y_bf16, int64_t M, int64_t N, int64_t K,
                        uint8_t* h_codes, uint8_t* h_scales, const float* t_h, cudaStream_t stream) {
   using namespace nvq::w4a4;
-  using GEO = Geo<PAIR>;
-  auto fn = nvfp4_gemm_kernel<EPI, PAIR>;
   CUtensorMap ma, mb, my;
   memset(&my, 0, sizeof(my));                               // EPI 1 never touches Y
   if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
                    BKB, BM) ||
       !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
-                   BKB, GEO::B_ROWS) ||
+                   BKB, BN) ||
       (EPI == 0 && !make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y_bf16, (uint64_t)N, (uint64_t)M,
                                 (uint64_t)N * 2, C_COLS, 32)))   // one epilogue warp: 32 rows x 64 columns
     return fail(NVQ_ERR_CUDA, "nvfp4_gemm_w4a4: tensor map encoding failed");
@@ -438,75 +434,34 @@ nvq_status launch_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, const fl
   p.M = (uint32_t)M;
   p.N = (uint32_t)N;
   p.K = (uint32_t)K;
-  p.num_m_tiles = (uint32_t)((M + GEO::TILE_M - 1) / GEO::TILE_M);
+  p.num_m_tiles = (uint32_t)((M + BM - 1) / BM);
   p.num_n_tiles = (uint32_t)((N + BN - 1) / BN);
   p.num_k_stages = (uint32_t)((K / 2 + BKB - 1) / BKB);
   p.k_atoms = (uint32_t)(K / 64);
   p.n_row_atoms = (uint32_t)((N + 127) / 128);
-  p.m_row_atoms = (uint32_t)((M + 127) / 128);
   // Sweep the smaller operand every wave (it stays in L2), stream the larger once.
   p.m_fastest = (uint64_t)M <= (uint64_t)N ? 1u : 0u;   // both operands have K/2 + K/16 bytes per row
   p.h_codes = h_codes;
   p.h_scales = h_scales;
   p.t_h = t_h;
   p.h_katoms = (uint32_t)(N / 2 / 64);
-  // The shared-memory opt-in (and the pair's cluster capacity) are per-device
-  // properties of the kernel: queried once per device.
+  // The shared-memory opt-in is a per-device setting of the kernel: once per device.
   int dev = 0;
   const cudaError_t de = cudaGetDevice(&dev);
   if (de != cudaSuccess) return cuda_fail(de, "nvfp4_gemm_w4a4: cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(NVQ_ERR_CUDA, "nvfp4_gemm_w4a4: device index out of range");
   static std::once_flag once[kMaxDevices];
   static cudaError_t attr_err[kMaxDevices];   // zero = cudaSuccess
-  static int max_units[kMaxDevices];          // resident CTAs (or CTA pairs)
-  std::call_once(once[dev], [dev, fn] {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, GEO::SMEM_BYTES);
-    int units = sm_count();
-    if (e == cudaSuccess && PAIR) {
-      cudaLaunchConfig_t q = {};
-      cudaLaunchAttribute at[1];
-      at[0].id = cudaLaunchAttributeClusterDimension;
-      at[0].val.clusterDim.x = 2;
-      at[0].val.clusterDim.y = 1;
-      at[0].val.clusterDim.z = 1;
-      q.gridDim = dim3(2, 1, 1);
-      q.blockDim = dim3(THREADS, 1, 1);
-      q.dynamicSmemBytes = GEO::SMEM_BYTES;
-      q.attrs = at;
-      q.numAttrs = 1;
-      e = cudaOccupancyMaxActiveClusters(&units, fn, &q);
-      if (e == cudaSuccess && units < 1) e = cudaErrorInvalidConfiguration;
-    }
-    attr_err[dev] = e;
-    max_units[dev] = units;
+  std::call_once(once[dev], [dev] {
+    attr_err[dev] = cudaFuncSetAttribute(nvfp4_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_BYTES);
   });
-  if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "nvfp4_gemm_w4a4: kernel attributes");
+  if (attr_err[dev] != cudaSuccess) return cuda_fail(attr_err[dev], "nvfp4_gemm_w4a4: smem attribute");
   const uint64_t tiles = (uint64_t)p.num_m_tiles * p.num_n_tiles;
-  const uint64_t units = std::min<uint64_t>(tiles, (uint64_t)max_units[dev]);
-  if constexpr (PAIR) {
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3((unsigned)(2 * units), 1, 1);
-    cfg.blockDim = dim3(THREADS, 1, 1);
-    cfg.dynamicSmemBytes = GEO::SMEM_BYTES;
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, fn, ma, mb, my, p);
-    if (e != cudaSuccess) return cuda_fail(e, "nvfp4_gemm_kernel launch");
-  } else {
-    fn<<<(unsigned)units, THREADS, GEO::SMEM_BYTES, stream>>>(ma, mb, my, p);
-  }
+  const int grid = (int)std::min<uint64_t>(tiles, (uint64_t)sm_count());
+  nvfp4_gemm_kernel<EPI><<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, my, p);
   return launch_status("nvfp4_gemm_kernel");
 }
-
-// CTA pairs (256 x 256 tiles) once the tile count fills the GPU; one CTA per
-// 128 x 256 tile for small M, where a pair tile would be mostly padding.
-bool w4a4_use_pairs(int64_t M) { return M > 256; }
 
 }  // namespace
 
@@ -526,11 +481,8 @@ nvq_status nvfp4_gemm_w4a4(const uint8_t* x_codes, const uint8_t* x_scales, cons
       !aligned16(y_bf16) || (reinterpret_cast<uintptr_t>(t_x) & 3u) || (reinterpret_cast<uintptr_t>(t_w) & 3u))
     return fail(NVQ_ERR_MISALIGNED, "nvfp4_gemm_w4a4: pointer not aligned");
   if (M == 0) return NVQ_OK;
-  if (w4a4_use_pairs(M))
-    return launch_w4a4<0, true>(x_codes, x_scales, t_x, w_codes, w_scales, t_w, y_bf16, M, N, K, nullptr, nullptr,
-                                nullptr, stream);
-  return launch_w4a4<0, false>(x_codes, x_scales, t_x, w_codes, w_scales, t_w, y_bf16, M, N, K, nullptr, nullptr,
-                               nullptr, stream);
+  return launch_w4a4<0>(x_codes, x_scales, t_x, w_codes, w_scales, t_w, y_bf16, M, N, K, nullptr, nullptr, nullptr,
+                        stream);
 }
 
 nvq_status nvfp4_gemm_w4a4_swiglu(const uint8_t* x_codes, const uint8_t* x_scales, const float* t_x,
@@ -550,11 +502,8 @@ nvq_status nvfp4_gemm_w4a4_swiglu(const uint8_t* x_codes, const uint8_t* x_scale
       (reinterpret_cast<uintptr_t>(t_w) & 3u) || (reinterpret_cast<uintptr_t>(t_h) & 3u))
     return fail(NVQ_ERR_MISALIGNED, "nvfp4_gemm_w4a4_swiglu: pointer not aligned");
   if (M == 0) return NVQ_OK;
-  if (w4a4_use_pairs(M))
-    return launch_w4a4<1, true>(x_codes, x_scales, t_x, w_codes, w_scales, t_w, nullptr, M, N, K, h_codes, h_scales,
-                                t_h, stream);
-  return launch_w4a4<1, false>(x_codes, x_scales, t_x, w_codes, w_scales, t_w, nullptr, M, N, K, h_codes, h_scales,
-                               t_h, stream);
+  return launch_w4a4<1>(x_codes, x_scales, t_x, w_codes, w_scales, t_w, nullptr, M, N, K, h_codes, h_scales, t_h,
+                        stream);
 }
 
 // ------------------------------------------------------------------ INT4
