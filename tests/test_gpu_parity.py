@@ -173,7 +173,9 @@ def test_gemm_tiny_case():
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 8, 64), (77, 136, 192), (200, 264, 320), (129, 520, 1024),
-                                   (300, 256, 4096), (256, 512, 256), (5, 1000, 128)])
+                                   (300, 256, 4096), (256, 512, 256), (5, 1000, 128),
+                                   (257, 520, 512), (513, 8, 256), (1000, 1000, 320), (300, 264, 64),
+                                   (640, 2048, 1024)])
 def test_gemm_ragged_shapes(M, N, K):
     x = synth.activations(M, K, seed=M + N + K)
     w = synth.weights(N, K, seed=M * N)
@@ -511,6 +513,7 @@ def _swiglu_case(M, I, K, seed, rows=None, t_scale=1.0, gpu_inputs=False):
 
 
 @pytest.mark.parametrize("M,I,K,t_scale", [(200, 256, 256, 1.0), (128, 384, 512, 1.0), (72, 128, 64, 1.0),
+                                           (300, 256, 256, 1.0), (520, 384, 320, 1.0),
                                            (130, 256, 320, 0.05), (64, 256, 256, 40.0)])
 def test_swiglu_gemm_emits_valid_nvfp4(M, I, K, t_scale):
     """Every block scale and code is the exact RTN result for some H' inside the
