@@ -162,7 +162,7 @@ __device__ __forceinline__ uint32_t quantize_block16(const float (&v)[16], float
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
   const uint32_t s = block_scale_code(amax, t, inv6t, tb.mid6);
   uint32_t w[2] = {0u, 0u};
-  if (tb.fast_ok[s]) {
+  if (__all_sync(0xFFFFFFFFu, tb.fast_ok[s] != 0u)) {        // warp-uniform: no warp runs both paths
     const float inv = tb.inv_d[s];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {                          // signed product: the sign lands on the code

@@ -18,10 +18,11 @@
 //     per CTA, the exact decision thresholds as bf16 values: the smallest bf16
 //     that lies above mu_i S t (or on it, when the tie goes up), found from
 //     h = fl(P t) and the exact residual e = fma(P, t, -h), P = mu_i S exact.
-//     The fast path (q = |x| * fl(1/fl(S t)), cvt.rn.satfinite.e2m1x2) is used
-//     for a scale code only if it gives the exact code on both sides of every
+//     The fast path (q = |x| * fl(1/fl(S t)), cvt.rn.satfinite.e2m1x2) is
+//     exact for a scale code if it gives the exact code on both sides of every
 //     threshold; both maps are monotone in |x|, so it is then exact for every
-//     bf16 input.  Other scale codes count thresholds with packed bf16x2
+//     bf16 input.  A warp takes it when it is exact for all 32 of its blocks'
+//     scale codes; otherwise the warp counts thresholds with packed bf16x2
 //     compares, which is exact by construction.
 #pragma once
 #include "ptx.cuh"
@@ -298,7 +299,10 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nvfp4_quantize_kernel(
     const float amax = bf16x2_hmax_to_f32(m2);
     const uint32_t s = block_scale_code(amax, t, inv6t, s_mid6);
     uint2 c;
-    if (s_fast_ok[s]) {
+    // Warp-uniform choice: the fast path only when it is exact for every
+    // block of the warp.  (Per-thread choice made nearly every warp run both
+    // paths, since a quarter to a third of the scale codes fail the fast check.)
+    if (__all_sync(0xFFFFFFFFu, s_fast_ok[s] != 0u)) {
       const float inv_d = s_inv_d[s];
       c.x = codes8_fast(w, inv_d);
       c.y = codes8_fast(w + 4, inv_d);
