@@ -212,6 +212,17 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nvfp4_quantize_kernel(
   __shared__ float s_mid6[128];                              // 6 x midpoints between E4M3 codes
   __shared__ uint16_t s_b[127][8];                           // thresholds while the tables are built
   __shared__ float s_t;
+  const uint32_t nblocks = rows * (K >> 4);                  // 16-element blocks, < 2^31 (checked on the host)
+  const uint32_t stride = gridDim.x * blockDim.x;
+  // Two blocks per thread stay in flight (this one and the next): their 64
+  // bytes are requested before t is known and the tables are built, so the
+  // first loads overlap that set-up and HBM latency overlaps the conversions.
+  uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0, q0 = p0, q1 = p0;
+  {
+    const uint32_t b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < nblocks) { p0 = __ldg(x + 2 * (size_t)b); p1 = __ldg(x + 2 * (size_t)b + 1); }
+    if (b + stride < nblocks) { q0 = __ldg(x + 2 * (size_t)(b + stride)); q1 = __ldg(x + 2 * (size_t)(b + stride) + 1); }
+  }
   if (threadIdx.x < 32) {
     float m = 0.f;
     if (t_in == nullptr)
@@ -268,28 +279,21 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nvfp4_quantize_kernel(
   const float inv6t = __frcp_rn(__fmul_rn(6.0f, t));
   const uint32_t nbk = K >> 4;                               // 16-element blocks per row
   const uint32_t atoms_per_rowtile = K >> 6;
-  const uint32_t nblocks = rows * nbk;                       // < 2^32 (checked on the host)
   const uint32_t lane = threadIdx.x & 31u;
-  const uint32_t stride = gridDim.x * blockDim.x;
   // (row, block-in-row) of this thread's block, advanced without a division.
   const uint32_t b0 = blockIdx.x * blockDim.x + threadIdx.x;
   uint32_t row = b0 / nbk, kb = b0 - row * nbk;
   const uint32_t step_r = stride / nbk, step_kb = stride - step_r * nbk;
-  // The next block's 32 bytes are requested before this one is processed, so
-  // the HBM latency of a tensor larger than L2 overlaps the conversion work.
-  uint4 p0 = make_uint4(0, 0, 0, 0), p1 = p0;
-  {
-    const uint32_t b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b < nblocks) { p0 = __ldg(x + 2 * (size_t)b); p1 = __ldg(x + 2 * (size_t)b + 1); }
-  }
   for (uint32_t base = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); base < nblocks; base += stride) {
     const uint32_t b = base + lane;
     const bool valid = b < nblocks;                          // nblocks % 4 == 0: groups of 4 agree
     uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    p0 = q0;
+    p1 = q1;
     {
-      const uint32_t bn = b + stride;                        // < 2^31 + one grid: no wrap
-      if (bn < nblocks) { p0 = __ldg(x + 2 * (size_t)bn); p1 = __ldg(x + 2 * (size_t)bn + 1); }
-      else { p0 = make_uint4(0, 0, 0, 0); p1 = p0; }
+      const uint32_t bn = b + 2 * stride;                    // < 2^31 + two grids: no wrap
+      if (bn < nblocks) { q0 = __ldg(x + 2 * (size_t)bn); q1 = __ldg(x + 2 * (size_t)bn + 1); }
+      else { q0 = make_uint4(0, 0, 0, 0); q1 = q0; }
     }
     uint32_t a[8];
 #pragma unroll
