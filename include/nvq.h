@@ -75,7 +75,12 @@ size_t nvq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 
 /* Synchronises `stream`, then reads and clears the device error word.
  * Returns NVQ_ERR_DEVICE_TIMEOUT if any kernel since the last check gave up on
- * a bounded wait, NVQ_ERR_CUDA if the synchronisation failed, else NVQ_OK. */
+ * a bounded wait, NVQ_ERR_CUDA if the synchronisation failed, else NVQ_OK.
+ * The error word is one per device and per loaded library, shared by every
+ * stream and every caller on that device: a timeout in a kernel on one stream
+ * is reported to whichever caller checks first (on any stream), and that
+ * check clears it for everyone.  Kernels still running on other streams are
+ * not waited for; a timeout they raise later is seen by a later check. */
 nvq_status nvq_check_device_error(void* stream);
 
 /* Diagnostic of the timeout path: launches one thread on `stream` that waits,
