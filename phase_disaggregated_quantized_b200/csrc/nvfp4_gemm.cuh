@@ -108,8 +108,10 @@ __device__ __forceinline__ void tile_coords(uint32_t tile, const Params& p, uint
 
 // ---------------------------------------------------------------- SiLU * mul -> NVFP4 epilogue
 // Per-CTA tables for the static tensor scale t_h of H, one entry per E4M3 block
-// scale code S: 1 / fl(S t_h), whether the fast map (fp32 product + cvt) gives
-// the exact RTN code for every fp32 input, and 6 x the midpoint to the next code.
+// scale code S: the multiplier of the fast map (1 / fl(S t_h), or that value
+// moved by 2^-20 relative, as for the activations), whether the fast map (fp32
+// product + cvt) gives the exact RTN code for every fp32 input, and 6 x the
+// midpoint to the next code.
 struct HTables {
   float inv_d[128];
   uint32_t fast_ok[128];
@@ -127,26 +129,38 @@ __device__ __forceinline__ uint32_t e2m1_code_f32(float x, float inv_d) {   // x
 __device__ __forceinline__ void build_h_table(HTables& tb, uint32_t c, float t) {
   const float S = e4m3_value(c);
   const float d = __fmul_rn(S, t);
-  const float inv = (c == 0) ? 0.f : __frcp_rn(d);
-  bool ok = (c == 0) || (d >= 1.17549435e-38f && !isinf(inv));
-  if (c != 0 && ok) {
-    for (int i = 0; i < 7 && ok; ++i) {
+  const float inv0 = (c == 0) ? 0.f : __frcp_rn(d);
+  float inv = inv0;
+  bool ok = (c == 0) || (d >= 1.17549435e-38f && !isinf(inv0));
+  auto exact_with = [&](float r) {
+    bool g = true;
+    for (int i = 0; i < 7 && g; ++i) {
       const float P = __fmul_rn(c_e2m1_mid[i], S);
       const float h = __fmul_rn(P, t);
       const float e = __fmaf_rn(P, t, -h);
       if (isinf(h)) {
-        ok = e2m1_code_f32(3.40282347e38f, inv) == (uint32_t)i;
+        g = e2m1_code_f32(3.40282347e38f, r) == (uint32_t)i;
         continue;
       }
       const bool pass_h = e < 0.f || (e == 0.f && ((i + 1) & 1) == 0);   // h above the threshold, or on a tie that goes up
       const uint32_t hb = __float_as_uint(h);
       const float x1 = pass_h ? h : __uint_as_float(hb + 1u);
-      if (e2m1_code_f32(x1, inv) != (uint32_t)(i + 1)) ok = false;
+      if (e2m1_code_f32(x1, r) != (uint32_t)(i + 1)) g = false;
       if (hb != 0u || !pass_h) {
         const float x0 = pass_h ? __uint_as_float(hb - 1u) : h;
-        if (e2m1_code_f32(x0, inv) != (uint32_t)i) ok = false;
+        if (e2m1_code_f32(x0, r) != (uint32_t)i) g = false;
       }
     }
+    return g;
+  };
+  if (c != 0 && ok) {                 // the multiplier candidates of the activation quantizer
+    const float cand[3] = {inv0, __fmul_rn(inv0, kNudgeDown), __fmul_rn(inv0, kNudgeUp)};
+    ok = false;
+    for (int j = 0; j < 3 && !ok; ++j)
+      if (!isinf(cand[j]) && exact_with(cand[j])) {
+        ok = true;
+        inv = cand[j];
+      }
   }
   tb.inv_d[c] = inv;
   tb.fast_ok[c] = ok ? 1u : 0u;

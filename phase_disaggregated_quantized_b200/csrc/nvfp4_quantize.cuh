@@ -18,12 +18,13 @@
 //     per CTA, the exact decision thresholds as bf16 values: the smallest bf16
 //     that lies above mu_i S t (or on it, when the tie goes up), found from
 //     h = fl(P t) and the exact residual e = fma(P, t, -h), P = mu_i S exact.
-//     The fast path (q = |x| * fl(1/fl(S t)), cvt.rn.satfinite.e2m1x2) is
-//     exact for a scale code if it gives the exact code on both sides of every
-//     threshold; both maps are monotone in |x|, so it is then exact for every
-//     bf16 input.  A warp takes it when it is exact for all 32 of its blocks'
-//     scale codes; otherwise the warp counts thresholds with packed bf16x2
-//     compares, which is exact by construction.
+//     The fast path (q = |x| * r, r = fl(1/fl(S t)) or that value moved by
+//     2^-20 relative, cvt.rn.satfinite.e2m1x2) is exact for a scale code if it
+//     gives the exact code on both sides of every threshold; both maps are
+//     monotone in |x|, so it is then exact for every bf16 input.  A warp takes
+//     it when it is exact for all 32 of its blocks' scale codes; otherwise the
+//     warp counts thresholds with packed bf16x2 compares, which is exact by
+//     construction.
 #pragma once
 #include "ptx.cuh"
 
@@ -119,6 +120,19 @@ __device__ __forceinline__ uint32_t e2m1x2_rn_satfinite(float hi, float lo) {
 }
 
 __constant__ float c_e2m1_mid[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
+
+// The fast map's multiplier r: fl(1/fl(S t)), or that value moved down or up
+// by 2^-20 relative when the plain one fails the exactness check.  With a
+// computed t = fl(amax / 2688), amax a bf16 value and 2688 = 2^7 * 21, every
+// threshold mu_i S t with mu_i S divisible by 21 lies within t's own rounding
+// error (<= 2^-24 relative) of a bf16 value, and on the same side of it for
+// every such threshold; the three roundings of the fast map (<= 3 * 2^-24)
+// then decide those inputs at random.  A 2^-20 move outweighs all of that and
+// puts every such input on one side, which is right for all of them in one of
+// the two directions, while thresholds that are not near a bf16 value keep
+// margins far above 2^-20.  The check decides in every case.
+constexpr float kNudgeDown = 1.0f - 0x1p-20f;
+constexpr float kNudgeUp = 1.0f + 0x1p-20f;
 
 // E4M3_RNE_satfinite(amax / (6 t)) decided on the exact quotient.  The estimate
 // amax * fl(1/fl(6t)) is within ~2 ulp, so the answer is s0 or a neighbour.
@@ -256,16 +270,27 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nvfp4_quantize_kernel(
 #pragma unroll
     for (int i = 0; i < 7; ++i) b[i] = s_b[c][i];
     const float d = __fmul_rn(S, t);
-    const float inv = (c == 0) ? 0.f : __frcp_rn(d);
-    bool ok = (c == 0) || (d >= 1.17549435e-38f && !isinf(inv));
+    const float inv0 = (c == 0) ? 0.f : __frcp_rn(d);
+    float inv = inv0;
+    bool ok = (c == 0) || (d >= 1.17549435e-38f && !isinf(inv0));
     if (c != 0 && ok) {
+      const float cand[3] = {inv0, __fmul_rn(inv0, kNudgeDown), __fmul_rn(inv0, kNudgeUp)};
+      ok = false;
+      for (int j = 0; j < 3 && !ok; ++j) {
+        if (isinf(cand[j])) continue;
+        bool g = true;
 #pragma unroll
-      for (int i = 0; i < 7; ++i) {
-        if (b[i] >= 0x7F80u) {
-          ok = ok && e2m1_fast_code(0x7F7Fu, inv) == (uint32_t)i;
-        } else {
-          ok = ok && e2m1_fast_code(b[i], inv) == (uint32_t)(i + 1);
-          if (b[i] > 0u) ok = ok && e2m1_fast_code(b[i] - 1u, inv) == (uint32_t)i;
+        for (int i = 0; i < 7; ++i) {
+          if (b[i] >= 0x7F80u) {
+            g = g && e2m1_fast_code(0x7F7Fu, cand[j]) == (uint32_t)i;
+          } else {
+            g = g && e2m1_fast_code(b[i], cand[j]) == (uint32_t)(i + 1);
+            if (b[i] > 0u) g = g && e2m1_fast_code(b[i] - 1u, cand[j]) == (uint32_t)i;
+          }
+        }
+        if (g) {
+          ok = true;
+          inv = cand[j];
         }
       }
     }

@@ -130,6 +130,22 @@ def test_quantize_decision_points_bit_exact(seed):
     assert_quant_parity(x)                   # and under the computed scale
 
 
+@pytest.mark.parametrize("amax", [87.0, 64.0, 162.0, 5.5, 127.5, 21.0, 1.0])
+def test_quantize_computed_scale_near_ties_bit_exact(amax):
+    """t = fl(amax / 2688) with amax a bf16 value: wherever mu_i S carries the
+    factor 21 (2688 = 2^7 * 21), the threshold mu_i S t lies within t's rounding
+    error of a bf16 value.  Elements on and one ulp around every mu_i S t, with
+    the tensor's max |x| pinned to amax so that the computed t is that one (21
+    gives an exact t and exact ties)."""
+    t = float(np.float32(np.float32(amax) / np.float32(2688.0)))
+    x = _decision_point_tensor(int(amax * 8) % 1000, t, rows=96, K=1024)
+    xf = x.float().clamp(-amax, amax)
+    xf[0, 0] = amax
+    x = xf.to(torch.bfloat16)
+    _, _, gt = assert_quant_parity(x)
+    assert float(gt.item()) == t
+
+
 def test_quantize_grid_round_trip():
     g = np.random.default_rng(4)
     rows, K = 8, 256
