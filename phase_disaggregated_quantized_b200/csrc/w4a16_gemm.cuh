@@ -23,9 +23,10 @@
 // k16 step j uses k = 32c + 4j + {0..3}: its 64-byte activation run feeds all
 // eight steps of both tiles of a dense unit.  Nibbles become bf16 (128 + u)
 // through the exponent bits.  The -136 offset (u - 8 = (128 + u) - 136) is
-// either subtracted in bf16 (exact) or, for up to two batch tiles, formed once per
-// unit as the chain -136 * sum(x) on the tensor core and passed as the C input
-// of both tiles' first MMA, so it costs no ALU work at all.  Each group's FP32
+// either subtracted in bf16 (exact; always so for 2:4-sparse units) or, for
+// dense units with up to two batch tiles, formed once per unit as the chain
+// -136 * sum(x) on the tensor core and passed as the C input of both tiles'
+// first MMA, so it costs no ALU work at all.  Each group's FP32
 // sum is scaled by the group's BF16 scale in FP32.
 //
 // Reduction.  A warp writes tiles it covered entirely straight to Y; the tiles
@@ -71,7 +72,7 @@ struct Cfg {
   static constexpr int XSLOT = (BARS + W * D * 8 + 15) / 16 * 16;   // 2 receive slots (pass parity)
   static constexpr int XBARS = XSLOT + 2 * TILEF * 4;    // receive-full [2], slot-free [2] barriers
   static constexpr int SMEM = XBARS + 32;
-  static constexpr bool ONES = NT8 <= 2;                 // -136 x through the tensor core
+  static constexpr bool ONES = NT8 <= 2;                 // dense units: -136 x through the tensor core
   static constexpr bool XDB = NT8 <= 2;                  // activations double-buffered one unit ahead
   static_assert(STAGE % 16 == 0 && (SG * U::CODE) % 16 == 0, "bulk-copy alignment");
   static_assert(W * 2 * TILEF * 4 <= RING, "warp partial tiles overlay the ring");
@@ -322,9 +323,13 @@ __device__ __forceinline__ void mma_sp_acc(float (&d)[4], const uint32_t (&a)[4]
 // activations k = 32 s + 16 (c / 2) + {0 .. 15}, of which words c % 2,
 // 2 + c % 2, 4 + c % 2, 6 + c % 2 feed its B fragment; the activations of a
 // step are loaded once for both tiles.  d[tt * NT8 + t] receives the group sum.
-template <int NT8, bool ONES>
+// The -136 offset is taken off each kept weight before the MMA (bf16x2
+// subtract, exact): the offset a dense unit gets from one -136 * sum(x) chain
+// would here need a second sparse MMA per step, since which activations meet
+// a kept weight depends on the row's metadata.
+template <int NT8>
 __device__ __forceinline__ void sparse_unit(uint32_t unit, uint32_t lane, const uint4* const (&xrow)[NT8],
-                                            const bool (&live)[NT8], uint32_t gk, float (&d)[2 * NT8][4]) {
+                                            uint32_t gk, float (&d)[2 * NT8][4]) {
   const uint32_t g = lane >> 2, c = lane & 3u, odd = c & 1u;
   uint32_t wsw[2][4], msw[2][4];
 #pragma unroll
@@ -334,8 +339,6 @@ __device__ __forceinline__ void sparse_unit(uint32_t unit, uint32_t lane, const 
     wsw[tt][0] = wq.x; wsw[tt][1] = wq.y; wsw[tt][2] = wq.z; wsw[tt][3] = wq.w;
     msw[tt][0] = mq.x; msw[tt][1] = mq.y; msw[tt][2] = mq.z; msw[tt][3] = mq.w;
   }
-  constexpr uint32_t kNeg136 = 0xC308C308u;
-  const uint32_t neg[4] = {kNeg136, kNeg136, kNeg136, kNeg136};
 #pragma unroll
   for (int t = 0; t < 2 * NT8; ++t)
 #pragma unroll
@@ -345,12 +348,8 @@ __device__ __forceinline__ void sparse_unit(uint32_t unit, uint32_t lane, const 
     uint32_t b[NT8][4];
 #pragma unroll
     for (int t = 0; t < NT8; ++t) {
-      uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
-      if (live[t]) {
-        const uint4* px = xrow[t] + gk * 16u + 4u * st + 2u * (c >> 1);
-        x0 = __ldg(px);
-        x1 = __ldg(px + 1);
-      }
+      const uint4* px = xrow[t] + gk * 16u + 4u * st + 2u * (c >> 1);   // rows >= M read row 0 (discarded)
+      const uint4 x0 = __ldg(px), x1 = __ldg(px + 1);
       b[t][0] = odd ? x0.y : x0.x;
       b[t][1] = odd ? x0.w : x0.z;
       b[t][2] = odd ? x1.y : x1.x;
@@ -360,15 +359,10 @@ __device__ __forceinline__ void sparse_unit(uint32_t unit, uint32_t lane, const 
     for (int tt = 0; tt < 2; ++tt) {
       uint32_t a[4];
       word_to_frag(wsw[tt][st], a);
-      if (!ONES) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) a[i] = bf16x2_sub136(a[i]);
-      }
+      for (int i = 0; i < 4; ++i) a[i] = bf16x2_sub136(a[i]);
 #pragma unroll
-      for (int t = 0; t < NT8; ++t) {
-        mma_sp_acc(d[tt * NT8 + t], a, b[t], msw[tt][st]);
-        if (ONES) mma_sp_acc(d[tt * NT8 + t], neg, b[t], msw[tt][st]);
-      }
+      for (int t = 0; t < NT8; ++t) mma_sp_acc(d[tt * NT8 + t], a, b[t], msw[tt][st]);
     }
   }
 }
@@ -472,16 +466,14 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
           for (int s = 0; s < D && irem > 0; ++s) issue();
         }
       }
-      // Activation rows of this lane (zero beyond M); for XDB two register
+      // Activation rows of this lane (row 0 beyond M: read, then discarded); for XDB two register
       // sets alternate between the unit being multiplied and the next one,
       // otherwise (the register budget of 4 batch tiles) each unit loads its own.
       const uint4* xrow[NT8];
-      bool live[NT8];
 #pragma unroll
       for (int t = 0; t < NT8; ++t) {
         const uint32_t m = m0 + 8 * t + gl;
-        live[t] = m < M;
-        xrow[t] = reinterpret_cast<const uint4*>(x + (size_t)(live[t] ? m : 0) * K + (SPARSE ? 0u : 32u * (lane & 3u)));
+        xrow[t] = reinterpret_cast<const uint4*>(x + (size_t)(m < M ? m : 0) * K + (SPARSE ? 0u : 32u * (lane & 3u)));
       }
       uint4 xa[NT8][4], xb[NT8][4];
 #pragma unroll
@@ -502,7 +494,7 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
           if ((uint32_t)i < n) {
             float d[NTT][4];
             if constexpr (SPARSE) {
-              sparse_unit<NT8, C::ONES>(stage + i * UC, lane, xrow, live, g + i, d);
+              sparse_unit<NT8>(stage + i * UC, lane, xrow, g + i, d);
             } else if constexpr (C::XDB) {
               uint4 (&cur)[NT8][4] = (i & 1) ? xb : xa;
               uint4 (&nxt)[NT8][4] = (i & 1) ? xa : xb;
