@@ -6,6 +6,7 @@
   python profile_case.py --op crossover --K 4096 --N 24576
   python profile_case.py --op streamed --M 8192 --layers 8
   python profile_case.py --op swiglu --M 8192 --K 4096 --N 24576
+  python profile_case.py --op library_nvfp4 --M 8192 --K 4096 --N 24576
 
 Inputs are drawn on the GPU from the seeded generators; the offline steps
 (weight quantization and reorder) run once before the measured calls.  The
@@ -29,7 +30,7 @@ from phase_disaggregated_quantized_b200 import synth  # noqa: E402
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=("gemm", "w4a16", "quantize", "crossover", "streamed", "swiglu"), required=True)
+    ap.add_argument("--op", choices=("gemm", "w4a16", "quantize", "crossover", "streamed", "swiglu", "library_nvfp4"), required=True)
     ap.add_argument("--layers", type=int, default=8, help="streamed: transformer layers of 4 Qwen3-8B linears")
     ap.add_argument("--M", type=int, default=0)
     ap.add_argument("--K", type=int, default=4096)
@@ -47,6 +48,8 @@ def main():
         return streamed(a, dev)
     if a.op == "swiglu":
         return swiglu(a, dev)
+    if a.op == "library_nvfp4":
+        return library_nvfp4(a, dev)
     x = synth.activations_cuda(a.M, a.K, seed=11, device=dev)
     if a.op == "gemm":
         w = synth.weights_cuda(a.N, a.K, seed=11, device=dev)
@@ -128,6 +131,30 @@ def _graph_time(run, iters):
     torch.cuda.synchronize()
     nvq.check_device_error()
     return e0.elapsed_time(e1) / 1e3 / iters
+
+
+def library_nvfp4(a, dev):
+    """Reference point, not part of the library: the same NVFP4 block-scaled GEMM
+    (16-element blocks, E4M3 scales, bf16 output) through the vendor library
+    (torch.nn.functional.scaled_mm, cuBLASLt), random codes, unit scales."""
+    import torch.nn.functional as F
+    M, K, N = a.M, a.K, a.N
+
+    def rup(v, m):
+        return (v + m - 1) // m * m
+    g = torch.Generator(device=dev).manual_seed(11)
+    xa = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g).view(torch.float4_e2m1fn_x2)
+    wb = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g).view(torch.float4_e2m1fn_x2)
+    one = 0x38                                                # E4M3 1.0
+    sa = torch.full((rup(M, 128) * rup(K // 16, 4),), one, dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
+    sb = torch.full((rup(N, 128) * rup(K // 16, 4),), one, dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
+
+    def run():
+        return F.scaled_mm(xa, wb.t(), sa, F.ScalingType.BlockWise1x16, sb, F.ScalingType.BlockWise1x16,
+                           swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                           output_dtype=torch.bfloat16)
+    s = _graph_time(run, a.iters)
+    print(f"library_nvfp4 M={M} K={K} N={N}: {1e6 * s:.2f} us/call, {2.0 * M * N * K / s / 1e12:.1f} TFLOP/s")
 
 
 def crossover(a, dev):
