@@ -2,7 +2,7 @@
 
   python profile_case.py --op gemm --M 8192 --K 4096 --N 24576
   python profile_case.py --op w4a16 --M 1 --K 4096 --N 24576
-  python profile_case.py --op quantize --M 8192 --K 12288
+  python profile_case.py --op quantize --M 8192 --K 12288 [--noalloc]
   python profile_case.py --op crossover --K 4096 --N 24576
   python profile_case.py --op streamed --M 8192 --layers 8
   python profile_case.py --op swiglu --M 8192 --K 4096 --N 24576
@@ -37,6 +37,7 @@ def main():
     ap.add_argument("--N", type=int, default=0)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--sparse", action="store_true", help="w4a16: the 2:4-sparse packed weights")
+    ap.add_argument("--noalloc", action="store_true", help="quantize: through nvfp4_quantize_noalloc")
     ap.add_argument("--copies", type=int, default=1,
                     help="w4a16: cycle through this many weight copies (a total above L2 gives cold-cache reads)")
     a = ap.parse_args()
@@ -85,7 +86,10 @@ def main():
         sc = torch.empty(nvq.nvfp4_scales_bytes(a.M, a.K), dtype=torch.uint8, device=dev)
         t = torch.empty(1, dtype=torch.float32, device=dev)
         ws = torch.empty(nvq.nvfp4_quantize_workspace_bytes(a.M, a.K), dtype=torch.uint8, device=dev)
-        run = lambda: nvq.nvfp4_quantize(x, None, codes=codes, scales=sc, tensor_scale_out=t, workspace=ws)  # noqa
+        if a.noalloc:                       # the entry point that keeps its scratch in the library
+            run = lambda: nvq.nvfp4_quantize_noalloc(x, None, codes=codes, scales=sc, tensor_scale_out=t)  # noqa
+        else:
+            run = lambda: nvq.nvfp4_quantize(x, None, codes=codes, scales=sc, tensor_scale_out=t, workspace=ws)  # noqa
         work = 2.0 * a.M * a.K * 2 + a.M * a.K * (0.5 + 1 / 16)
         unit = "GB/s"
     run()                                   # first call sets kernel attributes
