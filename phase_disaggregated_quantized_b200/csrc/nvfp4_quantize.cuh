@@ -60,6 +60,9 @@ __global__ void __launch_bounds__(kAmaxThreads) nvfp4_amax_kernel(const uint4* _
     m = bf16x2_max(m, bf16x2_max(bf16x2_max(vmax(v0), vmax(v1)), bf16x2_max(vmax(v2), vmax(v3))));
   }
   for (; i < nvec; i += stride) m = bf16x2_max(m, vmax(__ldg(x + i)));
+  // The quantize pass may start launching now (it waits for this grid before it
+  // reads the partials).
+  grid_launch_dependents();
   float f = bf16x2_hmax_to_f32(m);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
@@ -237,14 +240,18 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nvfp4_quantize_kernel(
     if (b < nblocks) { p0 = __ldg(x + 2 * (size_t)b); p1 = __ldg(x + 2 * (size_t)b + 1); }
     if (b + stride < nblocks) { q0 = __ldg(x + 2 * (size_t)(b + stride)); q1 = __ldg(x + 2 * (size_t)(b + stride) + 1); }
   }
+  // After the amax pass this kernel is launched early (programmatic dependent
+  // launch): x is only read by that pass, so the loads above may start during
+  // its tail, but its partials are read only after this wait (a no-op otherwise).
+  grid_dependency_wait();
   if (threadIdx.x < 32) {
     float m = 0.f;
     if (t_in == nullptr)
-      for (int i = threadIdx.x; i < npartial; i += 32) m = fmaxf(m, __ldg(partial + i));
+      for (int i = threadIdx.x; i < npartial; i += 32) m = fmaxf(m, __ldcg(partial + i));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if (threadIdx.x == 0) {
-      const float t = t_in != nullptr ? __ldg(t_in) : tensor_scale_of(m);
+      const float t = t_in != nullptr ? __ldcg(t_in) : tensor_scale_of(m);
       s_t = t;
       if (blockIdx.x == 0) *t_out = t;
     }

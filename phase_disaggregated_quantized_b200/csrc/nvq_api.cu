@@ -309,6 +309,34 @@ int amax_grid(int64_t rows, int64_t K) {
   return (int)std::max<size_t>(1, std::min<size_t>(nvq::kAmaxMaxBlocks, want));
 }
 
+// The quantize pass over rows x K.  Right after the amax pass of the same call
+// (after_amax) it is launched as a programmatic dependent of that pass: its CTAs
+// start and request their first blocks of x during the pass's tail and wait for
+// it before reading the partials.  Otherwise a plain launch (its x may come from
+// the kernel just before it).
+nvq_status launch_quantize_kernel(const void* x_bf16, int64_t rows, int64_t K, const float* tensor_scale_in,
+                                  const float* partial, int amax_blocks, uint8_t* codes, uint8_t* scales,
+                                  float* tensor_scale_out, bool after_amax, cudaStream_t stream) {
+  const uint64_t nblocks = (uint64_t)rows * (uint64_t)(K / 16);
+  const uint64_t want = (nblocks + nvq::kQuantThreads - 1) / nvq::kQuantThreads;
+  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count()));
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(nvq::kQuantThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_amax ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, nvq::nvfp4_quantize_kernel, static_cast<const uint4*>(x_bf16),
+                                           (uint32_t)rows, (uint32_t)K, tensor_scale_in, partial, amax_blocks,
+                                           reinterpret_cast<uint2*>(codes), scales, tensor_scale_out);
+  if (e != cudaSuccess) return cuda_fail(e, "nvfp4_quantize_kernel launch");
+  return launch_status("nvfp4_quantize_kernel");
+}
+
 // amax pre-pass (when t is not given) into `partial[0 .. amax_blocks)`, then the quantize pass.
 nvq_status quantize_launch(const void* x_bf16, int64_t rows, int64_t K, const float* tensor_scale_in, uint8_t* codes,
                            uint8_t* scales, float* tensor_scale_out, float* partial, int amax_blocks,
@@ -320,13 +348,8 @@ nvq_status quantize_launch(const void* x_bf16, int64_t rows, int64_t K, const fl
     nvq_status st = launch_status("nvfp4_amax_kernel");
     if (st != NVQ_OK) return st;
   }
-  const uint64_t nblocks = (uint64_t)rows * (uint64_t)(K / 16);
-  const uint64_t want = (nblocks + nvq::kQuantThreads - 1) / nvq::kQuantThreads;
-  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count()));
-  nvq::nvfp4_quantize_kernel<<<grid, nvq::kQuantThreads, 0, stream>>>(
-      static_cast<const uint4*>(x_bf16), (uint32_t)rows, (uint32_t)K, tensor_scale_in, partial, amax_blocks,
-      reinterpret_cast<uint2*>(codes), scales, tensor_scale_out);
-  return launch_status("nvfp4_quantize_kernel");
+  return launch_quantize_kernel(x_bf16, rows, K, tensor_scale_in, partial, amax_blocks, codes, scales,
+                                tensor_scale_out, amax_blocks > 0, stream);
 }
 
 }  // namespace
@@ -360,14 +383,8 @@ nvq_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, const flo
     nvq_status st = launch_status("nvfp4_amax_kernel");
     if (st != NVQ_OK) return st;
   }
-  const uint64_t nblocks = (uint64_t)rows * (uint64_t)(K / 16);
-  const uint64_t want = (nblocks + nvq::kQuantThreads - 1) / nvq::kQuantThreads;
-  const int grid = (int)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)sm_count()));
-  nvq::nvfp4_quantize_kernel<<<grid, nvq::kQuantThreads, 0, stream>>>(
-      static_cast<const uint4*>(x_bf16), (uint32_t)rows, (uint32_t)K, tensor_scale_in,
-      static_cast<const float*>(workspace), amax_blocks, reinterpret_cast<uint2*>(codes), scales,
-      tensor_scale_out);
-  return launch_status("nvfp4_quantize_kernel");
+  return launch_quantize_kernel(x_bf16, rows, K, tensor_scale_in, static_cast<const float*>(workspace),
+                                amax_blocks, codes, scales, tensor_scale_out, need_amax, stream);
 }
 
 nvq_status nvfp4_amax(const void* x_bf16, int64_t rows, int64_t K, float* amax_out, void* workspace,
