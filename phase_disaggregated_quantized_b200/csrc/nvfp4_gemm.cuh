@@ -352,7 +352,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     // A scale slot is free once the MMAs of the k-stage that used it (SF_SLOTS
     // k-stages back) have completed, i.e. once that stage's empty barrier has
     // fired: one commit per k-stage serves the TMA producer and these warps
-    // (a tcgen05.commit costs the MMA thread about as much as an MMA).
+    // (so the MMA thread commits once per k-stage, for both).
     uint32_t lag_stage = 0, lag_phase = 0, kg = 0;
     bool ok = true;
     for (uint32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
