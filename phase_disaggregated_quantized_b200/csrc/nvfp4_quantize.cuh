@@ -228,6 +228,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nvfp4_quantize_kernel(
   __shared__ uint4 s_thr[128];                               // 7 thresholds (bf16 bits) + pad
   __shared__ float s_mid6[128];                              // 6 x midpoints between E4M3 codes
   __shared__ uint16_t s_b[127][8];                           // thresholds while the tables are built
+  __shared__ uint8_t s_ck[127][8];                           // per threshold: which candidate multipliers pass
   __shared__ float s_t;
   const uint32_t nblocks = rows * (K >> 4);                  // 16-element blocks, < 2^31 (checked on the host)
   const uint32_t stride = gridDim.x * blockDim.x;
@@ -262,44 +263,53 @@ __global__ void __launch_bounds__(kQuantThreads, 1) nvfp4_quantize_kernel(
   // (fp32 quotient + cvt) provably agrees with them for every bf16 input: both
   // are monotone in |x|, so agreeing on both sides of every exact threshold
   // means agreeing everywhere.
-  // Thresholds first, one (code, midpoint) pair per thread ...
+  // One (code, midpoint) pair per thread: the exact threshold, and for each of
+  // the three candidate multipliers whether the fast map gives the exact code on
+  // both sides of it ...
   for (uint32_t i = threadIdx.x; i < 127u * 7u; i += blockDim.x) {
     const uint32_t c = i / 7u, j = i - 7u * c;
-    s_b[c][j] = c == 0 ? (uint16_t)0x7F80u
-                       : (uint16_t)e2m1_threshold_bits(__fmul_rn(c_e2m1_mid[j], e4m3_value(c)), t, (int)j);
+    uint32_t bits = 0x7F80u, pass = 0u;
+    if (c != 0) {
+      const float S = e4m3_value(c);
+      bits = e2m1_threshold_bits(__fmul_rn(c_e2m1_mid[j], S), t, (int)j);
+      const float inv0 = __frcp_rn(__fmul_rn(S, t));
+      const float cand[3] = {inv0, __fmul_rn(inv0, kNudgeDown), __fmul_rn(inv0, kNudgeUp)};
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        bool g = !isinf(cand[k]);
+        if (bits >= 0x7F80u) {
+          g = g && e2m1_fast_code(0x7F7Fu, cand[k]) == j;
+        } else {
+          g = g && e2m1_fast_code(bits, cand[k]) == j + 1u;
+          if (bits > 0u) g = g && e2m1_fast_code(bits - 1u, cand[k]) == j;
+        }
+        pass |= (g ? 1u : 0u) << k;
+      }
+    }
+    s_b[c][j] = (uint16_t)bits;
+    s_ck[c][j] = (uint8_t)pass;
   }
   __syncthreads();
-  // ... then one thread per code checks the fast path against them.
+  // ... then one thread per code takes the first candidate that passes all seven
+  // (the fast map is then exact for every bf16 input: both maps are monotone in |x|).
   if (threadIdx.x < 127) {
     const uint32_t c = threadIdx.x;
     const float S = e4m3_value(c);
-    uint32_t b[7];
+    uint32_t b[7], all = 7u;
 #pragma unroll
-    for (int i = 0; i < 7; ++i) b[i] = s_b[c][i];
+    for (int i = 0; i < 7; ++i) {
+      b[i] = s_b[c][i];
+      all &= s_ck[c][i];
+    }
     const float d = __fmul_rn(S, t);
     const float inv0 = (c == 0) ? 0.f : __frcp_rn(d);
     float inv = inv0;
     bool ok = (c == 0) || (d >= 1.17549435e-38f && !isinf(inv0));
     if (c != 0 && ok) {
-      const float cand[3] = {inv0, __fmul_rn(inv0, kNudgeDown), __fmul_rn(inv0, kNudgeUp)};
-      ok = false;
-      for (int j = 0; j < 3 && !ok; ++j) {
-        if (isinf(cand[j])) continue;
-        bool g = true;
-#pragma unroll
-        for (int i = 0; i < 7; ++i) {
-          if (b[i] >= 0x7F80u) {
-            g = g && e2m1_fast_code(0x7F7Fu, cand[j]) == (uint32_t)i;
-          } else {
-            g = g && e2m1_fast_code(b[i], cand[j]) == (uint32_t)(i + 1);
-            if (b[i] > 0u) g = g && e2m1_fast_code(b[i] - 1u, cand[j]) == (uint32_t)i;
-          }
-        }
-        if (g) {
-          ok = true;
-          inv = cand[j];
-        }
-      }
+      ok = all != 0u;
+      if (all & 1u) inv = inv0;
+      else if (all & 2u) inv = __fmul_rn(inv0, kNudgeDown);
+      else if (all & 4u) inv = __fmul_rn(inv0, kNudgeUp);
     }
     s_inv_d[c] = inv;
     s_fast_ok[c] = ok ? 1u : 0u;
