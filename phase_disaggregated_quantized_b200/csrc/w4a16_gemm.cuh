@@ -25,8 +25,10 @@
 // through the exponent bits.  The -136 offset (u - 8 = (128 + u) - 136) is
 // either subtracted in bf16 (exact; always so for 2:4-sparse units) or, for
 // dense units with up to two batch tiles, formed once per unit as the chain
-// -136 * sum(x) on the tensor core and passed as the C input of both tiles'
-// first MMA, so it costs no ALU work at all.  Each group's FP32
+// -136 * sum(x) on the tensor core: with two batch tiles passed as the C input
+// of both tiles' first MMA; with one, run independently of the weight chains
+// and added to their sums at the end (a shorter dependent path per unit).
+// Either way it costs no dequantization work.  Each group's FP32
 // sum is scaled by the group's BF16 scale in FP32.
 //
 // Reduction.  A warp writes tiles it covered entirely straight to Y; the tiles
@@ -61,7 +63,7 @@ struct Cfg {
   using U = Unit<SPARSE>;
   static constexpr int W = 8;                          // warps per CTA (two CTAs per SM)
   static constexpr int SG = 3;                         // units per ring stage
-  static constexpr int D = NT8 == 1 ? 2 : 4;           // ring stages per warp
+  static constexpr int D = NT8 == 1 ? 2 : 3;           // ring stages per warp (more shared memory leaves less L1 for x)
   static constexpr int THREADS = W * 32;
   static constexpr int MIN_CTAS = NT8 == 1 ? 2 : 1;     // CTAs per SM the register budget must allow
   static constexpr int STAGE = SG * U::BYTES;           // codes first, then the scales
@@ -74,6 +76,7 @@ struct Cfg {
   static constexpr int SMEM = XBARS + 32;
   static constexpr bool ONES = NT8 <= 2;                 // dense units: -136 x through the tensor core
   static constexpr bool XDB = NT8 <= 2;                  // activations double-buffered one unit ahead
+  static constexpr bool LATE = NT8 == 1;                  // -136 chain summed after the weight chains
   static_assert(STAGE % 16 == 0 && (SG * U::CODE) % 16 == 0, "bulk-copy alignment");
   static_assert(W * 2 * TILEF * 4 <= RING, "warp partial tiles overlay the ring");
   static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -254,7 +257,9 @@ __device__ __forceinline__ void store_tile(__nv_bfloat16* __restrict__ y, const 
 // One dense unit: 32 rows x 128 k, lane-major words.  LDS q (q = 0..3) of a
 // lane holds k16 steps 2q and 2q + 1 of MMA tiles 0 and 1: component
 // 2 (j & 1) + tt.  d[tt * NT8 + t] receives the group sum of tile tt, batch tile t.
-template <int NT8, bool ONES>
+// LATE: the weight chains start from zero, independent of the -136 chain, and
+// its sum is added at the end (a shorter dependent path per unit).
+template <int NT8, bool ONES, bool LATE>
 __device__ __forceinline__ void dense_unit(uint32_t addr, const uint4 (&xv)[NT8][4], float (&d)[2 * NT8][4]) {
   uint4 wq[4];
 #pragma unroll
@@ -292,7 +297,7 @@ __device__ __forceinline__ void dense_unit(uint32_t addr, const uint4 (&xv)[NT8]
       const uint4 q = xv[t][j >> 1];
       const uint32_t b0 = (j & 1) ? q.z : q.x, b1 = (j & 1) ? q.w : q.y;
       if (j == 0) {
-        if constexpr (ONES) {
+        if constexpr (ONES && !LATE) {
           mma_c(d[t], a0, b0, b1, offs[t]);
           mma_c(d[NT8 + t], a1, b0, b1, offs[t]);
         } else {
@@ -304,6 +309,12 @@ __device__ __forceinline__ void dense_unit(uint32_t addr, const uint4 (&xv)[NT8]
         mma_acc(d[NT8 + t], a1, b0, b1);
       }
     }
+  }
+  if constexpr (ONES && LATE) {
+#pragma unroll
+    for (int f = 0; f < 2 * NT8; ++f)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) d[f][e] += offs[f % NT8][e];
   }
 }
 
@@ -504,14 +515,14 @@ __global__ void __launch_bounds__(Cfg<NT8, SPARSE>::THREADS, Cfg<NT8, SPARSE>::M
 #pragma unroll
                 for (int v = 0; v < 4; ++v)
                   nxt[t][v] = __ldg(xrow[t] + gn * 16u + v);      // rows >= M read row 0 (discarded)
-              dense_unit<NT8, C::ONES>(stage + i * UC + lane * 16, cur, d);
+              dense_unit<NT8, C::ONES, C::LATE>(stage + i * UC + lane * 16, cur, d);
             } else {
 #pragma unroll
               for (int t = 0; t < NT8; ++t)
 #pragma unroll
                 for (int v = 0; v < 4; ++v)
                   xa[t][v] = __ldg(xrow[t] + (g + i) * 16u + v);
-              dense_unit<NT8, C::ONES>(stage + i * UC + lane * 16, xa, d);
+              dense_unit<NT8, C::ONES, C::LATE>(stage + i * UC + lane * 16, xa, d);
             }
             // Scale word tt of this lane: rows 16 tt + g (low half) and 16 tt + g + 8 (high half).
             uint32_t scw[TILES];
